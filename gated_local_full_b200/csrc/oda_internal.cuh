@@ -1,0 +1,159 @@
+// Internal definitions shared by liboda's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/oda.h"
+
+#define ODA_TILE 16  // tokens per paged block / ring tile
+
+struct oda_ctx {
+  oda_config cfg;
+  oda_layout_info lay;
+  int device;
+  int num_sms;
+  int attn_ctas_local;       // persistent grid of the Local attention kernel
+  int attn_ctas_full;        // persistent grid of the Full attention kernel
+  int max_parts;             // capacity of the partials buffer (in partials)
+  float* partials;           // [max_parts][G][d+2]
+  int* tickets;              // [max_batch * hkv], zero between launches
+  int* err;                  // device sticky error word
+  int* recall_tickets;       // recall-head split reduction counters
+  float* recall_partials;    // recall-head split partials
+  int recall_parts_cap;      // capacity of recall_partials in floats
+};
+
+namespace oda {
+
+// ----------------------------------------------------------------- host utils
+#define ODA_CUDA_TRY(expr)                                   \
+  do {                                                       \
+    cudaError_t _e = (expr);                                 \
+    if (_e != cudaSuccess) return ODA_ERR_CUDA;              \
+  } while (0)
+
+inline int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// ------------------------------------------------------------ device helpers
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void record_error(int* err, int code) {
+  if (err) atomicCAS(err, 0, code);
+}
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for phase `parity` of barrier `bar` to complete, giving up after
+// limit_ns nanoseconds of wall time. Returns false on timeout.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
+                                                  uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+  }
+}
+
+// One bulk (non-tensor) global->shared copy completing on an mbarrier.
+// dst, src 16-byte aligned; bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes,
+                                         uint32_t bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1], %2, [%3], %4;" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float fast_log2(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// bf16 pair (packed in a 32-bit word, low half first) -> two floats, exactly.
+__device__ __forceinline__ void bf16x2_to_f32(uint32_t w, float& lo, float& hi) {
+  lo = __uint_as_float(w << 16);
+  hi = __uint_as_float(w & 0xFFFF0000u);
+}
+
+}  // namespace oda
+
+// Host-side entry points implemented per translation unit (C++ linkage).
+namespace oda_impl {
+oda_status launch_append(oda_ctx* ctx, int lb, int le, const void* k_new, const void* v_new,
+                         const int32_t* seq_lens, const int32_t* block_table, void* kv_cache,
+                         void* ring, int B, cudaStream_t st);
+oda_status launch_ring_init(oda_ctx* ctx, int lb, int le, const int32_t* seq_lens,
+                            const int32_t* block_table, const void* kv_cache, void* ring, int B,
+                            cudaStream_t st);
+oda_status launch_attn(oda_ctx* ctx, bool ring_mode, int layer, const void* q,
+                       const int32_t* seq_lens, const void* kv, const int32_t* block_table,
+                       const int32_t* idx, const int32_t* count, void* out, float* lse, int B,
+                       cudaStream_t st);
+oda_status attn_setup(oda_ctx* ctx);
+oda_status launch_gate(oda_ctx* ctx, const float* scores, float theta, int B, uint8_t* flags,
+                       int32_t* idx, int32_t* count, cudaStream_t st,
+                       unsigned long long cond_handle, bool set_cond);
+oda_status launch_recall(oda_ctx* ctx, const void* h_prev, const void* emb, const void* h_local,
+                         int H, const void* W1, const float* b1, const float* w2, float b2,
+                         int hidden, float* scores, int B, cudaStream_t st);
+oda_status recall_setup(oda_ctx* ctx);
+oda_status launch_wait_selftest(oda_ctx* ctx, uint64_t timeout_ns, cudaStream_t st);
+}  // namespace oda_impl

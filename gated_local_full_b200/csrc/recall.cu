@@ -1,0 +1,443 @@
+// Recall head on the tensor cores.
+//
+// [SUM] Methodology: after Local, a recall score q_t = R_psi(h_{t-1}, E(x_t),
+// h^L_t) is computed from three states; [EXPL] Jargon / Recall head: a small
+// trained module (about 1.7 % of the backbone). The pages fix the inputs and
+// their order only; this library's head is
+//     score = w2 . GELU(W1 [h_{t-1}; E(x_t); h^L_t] + b1) + b2.
+//
+// Shape of the work: D[m][n] = sum_k W1[m][k] X[n][k] with M = hidden (4096),
+// N = batch (16), K = 3H (6144). The weight read (50 MB) bounds it; the MMA
+// only has to keep up, which CUDA-core FMAs at 16 rows per weight do not.
+//
+// B200 design:
+//   * the (m-tile, k-block) units are spread evenly over one CTA per SM
+//     (split-K, "stream-K" style), so 32 m-tiles still fill 148 SMs;
+//   * warp 0 streams 128x64 W1 tiles and N x64 X tiles with TMA (tensor maps,
+//     128-byte swizzle) into a ring of shared-memory stages; X is read from
+//     the three input tensors in place (three tensor maps, no concat copy);
+//   * warp 1 issues tcgen05.mma (kind::f16, bf16 in, f32 accumulate in TMEM,
+//     M = 128, N = batch rounded up to 16) and releases stages with
+//     tcgen05.commit;
+//   * warps 2..5 read the accumulator with tcgen05.ld. CTAs sharing an m-tile
+//     write partials; the last to take the m-tile's ticket sums them in a
+//     fixed order, adds b1, applies GELU and the w2 dot product; the last
+//     m-tile sums the per-tile dot products in order and adds b2. The result
+//     is deterministic run to run.
+#include <cuda.h>
+
+#include "oda_internal.cuh"
+
+using namespace oda;
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;                 // 64 bf16 = one 128-byte swizzle row
+constexpr int A_STAGE_BYTES = BM * BK * 2;
+constexpr int MAX_N = 256;
+constexpr int MAX_MT = 64;             // hidden <= 8192
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+struct RecallArgs {
+  const float* b1;
+  const float* w2;
+  float b2;
+  float* scores;
+  float* partials;   // [P + MT][N][128]
+  float* spart;      // [MT][N]
+  int* tickets;      // [MT] per m-tile, [MAX_MT] for the final sum
+  int* err;
+  int B, N, MT, KB, H, stages;
+};
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
+// 1024 bytes apart (SBO), leading offset unused (1), descriptor version 1.
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1u << 16;
+  d |= (uint64_t)(1024u >> 4) << 32;
+  d |= (uint64_t)1u << 46;
+  d |= (uint64_t)2u << 61;
+  return d;
+}
+
+// Instruction descriptor: kind::f16, bf16 A and B (K-major), f32 D, M=128.
+__host__ __device__ constexpr uint32_t umma_idesc_bf16(int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) |
+         ((uint32_t)(BM >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void fence_before_sync() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void fence_after_sync() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void epi_bar() {  // named barrier over the 4 epilogue warps
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+
+__device__ __forceinline__ float gelu_erf(float u) {
+  return 0.5f * u * (1.0f + erff(u * 0.70710678118654752f));
+}
+
+__global__ void __launch_bounds__(192, 1)
+recall_kernel(const __grid_constant__ CUtensorMap tm_w1, const __grid_constant__ CUtensorMap tm_x0,
+              const __grid_constant__ CUtensorMap tm_x1, const __grid_constant__ CUtensorMap tm_x2,
+              const RecallArgs a) {
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw = smem_addr(smem_raw);
+  const uint32_t pad = ((raw + 1023u) & ~1023u) - raw;
+  unsigned char* smem = smem_raw + pad;
+  const int S = a.stages;
+  const int N = a.N;
+  const uint32_t b_stage_bytes = (uint32_t)N * BK * 2;
+  unsigned char* sa = smem;
+  unsigned char* sb = sa + (size_t)S * A_STAGE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sb + (size_t)S * b_stage_bytes);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + S;
+  uint64_t* acc_full = bars + 2 * S;
+  uint64_t* acc_empty = acc_full + 1;
+  uint64_t* done_bar = acc_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 3);
+  int* sflag = reinterpret_cast<int*>(tmem_slot + 1);
+  float* red = reinterpret_cast<float*>(sflag + 4);  // [4][MAX_N]
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int U = a.MT * a.KB;
+  const int P = (int)gridDim.x;
+  const int c = (int)blockIdx.x;
+  const int u0 = (int)(((long long)c * U) / P);
+  const int u1 = (int)(((long long)(c + 1) * U) / P);
+  uint32_t ncols = 32;
+  while ((int)ncols < N) ncols <<= 1;
+
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(smem_addr(&full[s]), 1);
+      mbar_init(smem_addr(&empty[s]), 1);
+    }
+    mbar_init(smem_addr(acc_full), 1);
+    mbar_init(smem_addr(acc_empty), 4);
+    mbar_init(smem_addr(done_bar), 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    __syncwarp();
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_addr(tmem_slot)),
+                 "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+
+  if (u0 < u1) {
+    if (warp == 0) {
+      // ------------------------------------------------------ TMA producer
+      if (lane == 0) {
+        const uint32_t tx = A_STAGE_BYTES + b_stage_bytes;
+        for (int u = u0, i = 0; u < u1; ++u, ++i) {
+          const int s = i % S;
+          const uint32_t par = (uint32_t)(((i / S) & 1) ^ 1);
+          if (!mbar_wait_bounded(smem_addr(&empty[s]), par, kWaitLimitNs)) {
+            record_error(a.err, ODA_ERR_TIMEOUT);
+            break;
+          }
+          const int mt = u / a.KB, kb = u % a.KB;
+          const uint32_t fb = smem_addr(&full[s]);
+          mbar_arrive_expect_tx(fb, tx);
+          tma_load_2d(smem_addr(sa + (size_t)s * A_STAGE_BYTES), &tm_w1, kb * BK, mt * BM, fb);
+          const int kglob = kb * BK;
+          const int seg = kglob / a.H;
+          const int kin = kglob - seg * a.H;
+          const CUtensorMap* xm = seg == 0 ? &tm_x0 : (seg == 1 ? &tm_x1 : &tm_x2);
+          tma_load_2d(smem_addr(sb + (size_t)s * b_stage_bytes), xm, kin, 0, fb);
+        }
+      }
+    } else if (warp == 1) {
+      // ------------------------------------------------------- MMA issuer
+      if (lane == 0) {
+        const uint32_t idesc = umma_idesc_bf16(N);
+        int i = 0, j = 0;
+        bool ok = true;
+        for (int u = u0; u < u1 && ok; ++j) {
+          const int mt = u / a.KB;
+          const int uend = min(u1, (mt + 1) * a.KB);
+          if (j > 0 && !mbar_wait_bounded(smem_addr(acc_empty), (uint32_t)((j - 1) & 1),
+                                          kWaitLimitNs)) {
+            record_error(a.err, ODA_ERR_TIMEOUT);
+            break;
+          }
+          fence_after_sync();
+          for (; u < uend; ++u, ++i) {
+            const int s = i % S;
+            if (!mbar_wait_bounded(smem_addr(&full[s]), (uint32_t)((i / S) & 1), kWaitLimitNs)) {
+              record_error(a.err, ODA_ERR_TIMEOUT);
+              ok = false;
+              break;
+            }
+            fence_after_sync();
+            const uint64_t ad = umma_desc_sw128(smem_addr(sa + (size_t)s * A_STAGE_BYTES));
+            const uint64_t bd = umma_desc_sw128(smem_addr(sb + (size_t)s * b_stage_bytes));
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              // +32 bytes per 16-element K step inside the swizzled row
+              umma_bf16(tmem, ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), idesc,
+                        (u == max(u0, mt * a.KB) && kk == 0) ? 0u : 1u);
+            }
+            umma_commit(smem_addr(&empty[s]));
+          }
+          if (ok) umma_commit(smem_addr(acc_full));
+        }
+        umma_commit(smem_addr(done_bar));
+      }
+    } else {
+      // ------------------------------------------------------- epilogue
+      const int q = warp & 3;              // TMEM lane quarter this warp may read
+      const int m = q * 32 + lane;         // row of the m-tile
+      const int ew = warp - 2;             // 0..3
+      int j = 0;
+      for (int u = u0; u < u1; ++j) {
+        const int mt = u / a.KB;
+        const int seg_lo = mt * a.KB, seg_hi = (mt + 1) * a.KB;
+        const int uend = min(u1, seg_hi);
+        u = uend;
+        // one elected waiter so that all four epilogue warps agree on the outcome
+        if (tid == 64) {
+          const bool got = mbar_wait_bounded(smem_addr(acc_full), (uint32_t)(j & 1), kWaitLimitNs);
+          if (!got) record_error(a.err, ODA_ERR_TIMEOUT);
+          sflag[2] = got ? 1 : 0;
+        }
+        epi_bar();
+        if (!sflag[2]) break;
+        fence_after_sync();
+        const int c_first = (int)(((long long)(seg_lo + 1) * P - 1) / U);
+        const int c_last = (int)(((long long)seg_hi * P - 1) / U);
+        const int nparts = c_last - c_first + 1;
+        float* mypart = a.partials + (size_t)(c + mt) * N * BM;
+        // TMEM -> registers -> partials (always written; the merge reads them)
+        for (int n0 = 0; n0 < N; n0 += 16) {
+          float v[16];
+          tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)n0, v);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) mypart[(size_t)(n0 + e) * BM + m] = v[e];
+        }
+        fence_before_sync();
+        if (lane == 0) mbar_arrive(smem_addr(acc_empty));
+        epi_bar();
+        bool last = true;
+        if (nparts > 1) {
+          if (tid == 64) {
+            __threadfence();
+            const int prev = atomicAdd(&a.tickets[mt], 1);
+            sflag[0] = (prev == nparts - 1) ? 1 : 0;
+          }
+          epi_bar();
+          last = sflag[0] != 0;
+          epi_bar();
+        }
+        if (last) {
+          __threadfence();
+          const float bias = a.b1[mt * BM + m];
+          const float wo = a.w2[mt * BM + m];
+          for (int n = 0; n < N; ++n) {
+            float acc = 0.f;
+            for (int c2 = c_first; c2 <= c_last; ++c2)
+              acc += __ldcg(a.partials + ((size_t)(c2 + mt) * N + n) * BM + m);
+            float contrib = wo * gelu_erf(acc + bias);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) contrib += __shfl_xor_sync(0xffffffffu, contrib, o);
+            if (lane == 0) red[ew * MAX_N + n] = contrib;
+          }
+          epi_bar();
+          for (int n = tid - 64; n < N; n += 128) {
+            // fixed order over the four row quarters: rows 0-31, 32-63, 64-95, 96-127
+            float s = 0.f;
+            for (int qq = 0; qq < 4; ++qq) s += red[((qq + 2) & 3) * MAX_N + n];
+            a.spart[(size_t)mt * N + n] = s;
+          }
+          if (tid == 64) a.tickets[mt] = 0;
+          epi_bar();
+          if (tid == 64) {
+            __threadfence();
+            const int prev = atomicAdd(&a.tickets[MAX_MT], 1);
+            sflag[1] = (prev == a.MT - 1) ? 1 : 0;
+          }
+          epi_bar();
+          if (sflag[1]) {
+            __threadfence();
+            for (int n = tid - 64; n < a.B; n += 128) {
+              float s = 0.f;
+              for (int t2 = 0; t2 < a.MT; ++t2) s += __ldcg(a.spart + (size_t)t2 * N + n);
+              a.scores[n] = s + a.b2;
+            }
+            if (tid == 64) a.tickets[MAX_MT] = 0;
+          }
+          epi_bar();
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    __syncwarp();
+    // all MMAs of this CTA must have completed before TMEM is released
+    if (u0 < u1) {
+      if (!mbar_wait_bounded(smem_addr(done_bar), 0u, kWaitLimitNs) && lane == 0)
+        record_error(a.err, ODA_ERR_TIMEOUT);
+    }
+    __syncwarp();
+    fence_after_sync();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(ncols)
+                 : "memory");
+  }
+}
+
+// ------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encoder() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+bool encode_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_in,
+               uint32_t box_out) {
+  EncodeTiledFn enc = get_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {box_in, box_out};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int stages_for(int n) {
+  const int per = A_STAGE_BYTES + n * BK * 2;
+  int s = (200 * 1024) / per;
+  if (s > 8) s = 8;
+  if (s < 2) s = 2;
+  return s;
+}
+
+size_t smem_for(int n, int s) {
+  return 1024 + (size_t)s * (A_STAGE_BYTES + n * BK * 2) + (size_t)(2 * s + 3) * 8 + 4 + 16 +
+         4 * MAX_N * 4 + 64;
+}
+
+}  // namespace
+
+namespace oda_impl {
+
+oda_status recall_setup(oda_ctx* ctx) {
+  const size_t max_smem = smem_for(MAX_N, stages_for(MAX_N));
+  size_t best = max_smem;
+  for (int n = 16; n <= MAX_N; n += 16) best = best > smem_for(n, stages_for(n)) ? best : smem_for(n, stages_for(n));
+  ODA_CUDA_TRY(cudaFuncSetAttribute(recall_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)best));
+  const size_t pfl = (size_t)(ctx->num_sms + MAX_MT) * MAX_N * BM + (size_t)MAX_MT * MAX_N;
+  ODA_CUDA_TRY(cudaMalloc(&ctx->recall_partials, pfl * sizeof(float)));
+  ctx->recall_parts_cap = (int)((size_t)(ctx->num_sms + MAX_MT) * MAX_N * BM);
+  ODA_CUDA_TRY(cudaMalloc(&ctx->recall_tickets, (MAX_MT + 1) * sizeof(int)));
+  ODA_CUDA_TRY(cudaMemset(ctx->recall_tickets, 0, (MAX_MT + 1) * sizeof(int)));
+  return ODA_OK;
+}
+
+oda_status launch_recall(oda_ctx* ctx, const void* h_prev, const void* emb, const void* h_local,
+                         int H, const void* W1, const float* b1, const float* w2, float b2,
+                         int hidden, float* scores, int B, cudaStream_t st) {
+  if (B < 1 || B > MAX_N || H < BK || H % BK != 0 || hidden < BM || hidden % BM != 0 ||
+      hidden / BM > MAX_MT)
+    return ODA_ERR_SHAPE;
+  const int N = ((B + 15) / 16) * 16;
+  CUtensorMap tw, t0, t1, t2;
+  const uint64_t K = 3ull * (uint64_t)H;
+  if (!encode_2d(&tw, W1, K, (uint64_t)hidden, BK, BM)) return ODA_ERR_CUDA;
+  if (!encode_2d(&t0, h_prev, (uint64_t)H, (uint64_t)B, BK, (uint32_t)N)) return ODA_ERR_CUDA;
+  if (!encode_2d(&t1, emb, (uint64_t)H, (uint64_t)B, BK, (uint32_t)N)) return ODA_ERR_CUDA;
+  if (!encode_2d(&t2, h_local, (uint64_t)H, (uint64_t)B, BK, (uint32_t)N)) return ODA_ERR_CUDA;
+  RecallArgs a;
+  a.b1 = b1;
+  a.w2 = w2;
+  a.b2 = b2;
+  a.scores = scores;
+  a.partials = ctx->recall_partials;
+  a.spart = ctx->recall_partials + ctx->recall_parts_cap;
+  a.tickets = ctx->recall_tickets;
+  a.err = ctx->err;
+  a.B = B;
+  a.N = N;
+  a.MT = hidden / BM;
+  a.KB = (int)(K / BK);
+  a.H = H;
+  a.stages = stages_for(N);
+  const int U = a.MT * a.KB;
+  const int grid = U < ctx->num_sms ? U : ctx->num_sms;
+  recall_kernel<<<grid, 192, smem_for(N, a.stages), st>>>(tw, t0, t1, t2, a);
+  return cudaGetLastError() == cudaSuccess ? ODA_OK : ODA_ERR_CUDA;
+}
+
+}  // namespace oda_impl

@@ -1,0 +1,190 @@
+// One decode step: plain launches, or a CUDA graph with a device-side IF node.
+//
+// [SUM] Methodology / Local-First Decoding gives the order: commit the token,
+// run Local, score, and recompute with Full only if q_t > theta.
+// [SUM] Efficient Execution: the runtime uses GPU-side conditional CUDA
+// graphs, so the decision never returns to the host. Here the gate kernel
+// writes the IF node's condition (count > 0); with no flagged row the graph
+// launches no Full kernel at all.
+#include <stdlib.h>
+
+#include "oda_internal.cuh"
+
+struct oda_graph {
+  oda_ctx* ctx;
+  cudaGraph_t graph;
+  cudaGraphExec_t exec;
+};
+
+namespace {
+
+oda_status check_desc(const oda_ctx* ctx, const oda_step_desc* d) {
+  if (!ctx || !d) return ODA_ERR_ARG;
+  if (d->B < 1) return ODA_ERR_ARG;
+  if (d->B > ctx->cfg.max_batch) return ODA_ERR_SHAPE;
+  if (!d->q || !d->k_new || !d->v_new || !d->seq_lens || !d->block_table || !d->kv_cache ||
+      !d->ring || !d->out || !d->flags || !d->idx || !d->count)
+    return ODA_ERR_ARG;
+  if (d->W1 && (!d->h_prev || !d->emb || !d->h_local || !d->b1 || !d->w2 || !d->scores))
+    return ODA_ERR_ARG;
+  if (!d->W1 && !d->gate_scores && !d->scores) return ODA_ERR_ARG;
+  return ODA_OK;
+}
+
+size_t layer_elems(const oda_ctx* ctx, int B, int heads) {
+  return (size_t)B * heads * ctx->cfg.head_dim;
+}
+
+oda_status pre_part(oda_ctx* ctx, const oda_step_desc* d, cudaStream_t st,
+                    unsigned long long cond, bool set_cond) {
+  const oda_config& c = ctx->cfg;
+  const size_t eb = (size_t)ctx->lay.elem_bytes;
+  oda_status s = oda_impl::launch_append(ctx, 0, c.layers, d->k_new, d->v_new, d->seq_lens,
+                                         d->block_table, d->kv_cache, d->ring, d->B, st);
+  if (s != ODA_OK) return s;
+  for (int l = 0; l < c.layers; ++l) {
+    const size_t qo = (size_t)l * layer_elems(ctx, d->B, c.hq) * eb;
+    float* lse = d->lse ? d->lse + (size_t)l * d->B * c.hq : nullptr;
+    s = oda_impl::launch_attn(ctx, true, l, static_cast<const char*>(d->q) + qo, d->seq_lens,
+                              d->ring, nullptr, nullptr, nullptr,
+                              static_cast<char*>(d->out) + qo, lse, d->B, st);
+    if (s != ODA_OK) return s;
+  }
+  if (d->W1) {
+    s = oda_impl::launch_recall(ctx, d->h_prev, d->emb, d->h_local, d->H, d->W1, d->b1, d->w2,
+                                d->b2, d->hidden, d->scores, d->B, st);
+    if (s != ODA_OK) return s;
+  }
+  const float* gs = d->gate_scores ? d->gate_scores : d->scores;
+  return oda_impl::launch_gate(ctx, gs, d->theta, d->B, d->flags, d->idx, d->count, st, cond,
+                               set_cond);
+}
+
+oda_status full_part(oda_ctx* ctx, const oda_step_desc* d, cudaStream_t st) {
+  const oda_config& c = ctx->cfg;
+  const size_t eb = (size_t)ctx->lay.elem_bytes;
+  for (int l = 0; l < c.layers; ++l) {
+    const size_t qo = (size_t)l * layer_elems(ctx, d->B, c.hq) * eb;
+    float* lse = d->lse ? d->lse + (size_t)l * d->B * c.hq : nullptr;
+    oda_status s = oda_impl::launch_attn(ctx, false, l, static_cast<const char*>(d->q) + qo,
+                                         d->seq_lens, d->kv_cache, d->block_table, d->idx,
+                                         d->count, static_cast<char*>(d->out) + qo, lse, d->B, st);
+    if (s != ODA_OK) return s;
+  }
+  return ODA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+oda_status oda_step_run(oda_ctx* ctx, const oda_step_desc* d, oda_stream stream) {
+  oda_status s = check_desc(ctx, d);
+  if (s != ODA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  s = pre_part(ctx, d, st, 0ull, false);
+  if (s != ODA_OK) return s;
+  return full_part(ctx, d, st);
+}
+
+oda_status oda_step_graph_create(oda_ctx* ctx, const oda_step_desc* d, oda_graph** out) {
+  if (!out) return ODA_ERR_ARG;
+  *out = nullptr;
+  oda_status s = check_desc(ctx, d);
+  if (s != ODA_OK) return s;
+  cudaStream_t st = nullptr, st2 = nullptr;
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t exec = nullptr;
+  ODA_CUDA_TRY(cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking));
+  if (cudaStreamCreateWithFlags(&st2, cudaStreamNonBlocking) != cudaSuccess) {
+    cudaStreamDestroy(st);
+    return ODA_ERR_CUDA;
+  }
+  s = ODA_ERR_CUDA;
+  do {
+    if (cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal) != cudaSuccess) break;
+    cudaStreamCaptureStatus cs;
+    cudaGraph_t cap = nullptr;
+    const cudaGraphNode_t* deps = nullptr;
+    size_t ndeps = 0;
+    cudaGraphConditionalHandle handle = 0;
+    bool ok = cudaStreamGetCaptureInfo(st, &cs, nullptr, &cap, &deps, &ndeps) == cudaSuccess &&
+              cs == cudaStreamCaptureStatusActive &&
+              cudaGraphConditionalHandleCreate(&handle, cap, 0, cudaGraphCondAssignDefault) ==
+                  cudaSuccess;
+    oda_status ps = ok ? pre_part(ctx, d, st, (unsigned long long)handle, true) : ODA_ERR_CUDA;
+    cudaGraphNode_t cond_node = nullptr;
+    cudaGraph_t body = nullptr;
+    if (ps == ODA_OK &&
+        cudaStreamGetCaptureInfo(st, &cs, nullptr, &cap, &deps, &ndeps) == cudaSuccess) {
+      cudaGraphNodeParams p = {};
+      p.type = cudaGraphNodeTypeConditional;
+      p.conditional.handle = handle;
+      p.conditional.type = cudaGraphCondTypeIf;
+      p.conditional.size = 1;
+      if (cudaGraphAddNode(&cond_node, cap, deps, ndeps, &p) == cudaSuccess) {
+        body = p.conditional.phGraph_out[0];
+        ok = cudaStreamUpdateCaptureDependencies(st, &cond_node, 1,
+                                                 cudaStreamSetCaptureDependencies) == cudaSuccess;
+      } else {
+        ok = false;
+      }
+    } else {
+      ok = false;
+    }
+    if (ok) {
+      ok = cudaStreamBeginCaptureToGraph(st2, body, nullptr, nullptr, 0,
+                                         cudaStreamCaptureModeThreadLocal) == cudaSuccess;
+      if (ok) {
+        const oda_status fs = full_part(ctx, d, st2);
+        cudaGraph_t body_out = nullptr;
+        ok = cudaStreamEndCapture(st2, &body_out) == cudaSuccess && fs == ODA_OK;
+      }
+    }
+    cudaGraph_t done = nullptr;
+    const bool ended = cudaStreamEndCapture(st, &done) == cudaSuccess;
+    if (!ok || !ended || ps != ODA_OK) {
+      if (done) cudaGraphDestroy(done);
+      s = ps != ODA_OK ? ps : ODA_ERR_CUDA;
+      break;
+    }
+    graph = done;
+    if (cudaGraphInstantiate(&exec, graph, 0) != cudaSuccess) {
+      cudaGraphDestroy(graph);
+      graph = nullptr;
+      break;
+    }
+    s = ODA_OK;
+  } while (false);
+  cudaGetLastError();
+  cudaStreamDestroy(st);
+  cudaStreamDestroy(st2);
+  if (s != ODA_OK) return s;
+  oda_graph* g = static_cast<oda_graph*>(calloc(1, sizeof(oda_graph)));
+  if (!g) {
+    cudaGraphExecDestroy(exec);
+    cudaGraphDestroy(graph);
+    return ODA_ERR_ARG;
+  }
+  g->ctx = ctx;
+  g->graph = graph;
+  g->exec = exec;
+  *out = g;
+  return ODA_OK;
+}
+
+oda_status oda_step_graph_launch(oda_graph* g, oda_stream stream) {
+  if (!g || !g->exec) return ODA_ERR_ARG;
+  ODA_CUDA_TRY(cudaGraphLaunch(g->exec, static_cast<cudaStream_t>(stream)));
+  return ODA_OK;
+}
+
+oda_status oda_step_graph_destroy(oda_graph* g) {
+  if (!g) return ODA_OK;
+  if (g->exec) cudaGraphExecDestroy(g->exec);
+  if (g->graph) cudaGraphDestroy(g->graph);
+  free(g);
+  return ODA_OK;
+}
+
+}  // extern "C"

@@ -331,11 +331,18 @@ def recall_step(ctx: int, batch: int = 16) -> Workload:
                     t0=np.full(batch, ctx, np.int64), steps=1, seed=4, recall=True)
 
 
-def custom(name: str, *, dtype="bf16", layers=1, batch=2, hq=4, hkv=2, d=128, sink=4,
+def custom(name: str, *, dtype="bf16", layers=1, batch=None, hq=4, hkv=2, d=128, sink=4,
            window=64, block_size=16, t0=(100, 37), steps=1, seed=11, sigma_kv=0.5,
            flag_rate=None, flag_per="row", fixed_scores=None, recall=False, hidden=2048,
            recall_hidden=4096) -> Workload:
     """Free-form workload for edge cases (ragged tails, t <= s+w, tiny windows)."""
+    t0 = np.asarray(t0, np.int64).reshape(-1)
+    if batch is None:
+        batch = int(t0.size)
+    if t0.size == 1 and batch > 1:
+        t0 = np.repeat(t0, batch)
+    if t0.size != batch:
+        raise ValueError("t0 needs one context length per row")
     return Workload(name=name, dtype=dtype, layers=layers, batch=batch, hq=hq, hkv=hkv, d=d,
                     sink=sink, window=window, block_size=block_size,
                     t0=np.asarray(t0, np.int64), steps=steps, seed=seed, sigma_kv=sigma_kv,
