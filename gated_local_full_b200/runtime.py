@@ -1,12 +1,14 @@
 """Decode-step runtime: static buffers + one captured CUDA graph per step.
 
 A serving loop writes each step's inputs (queries, the new token's K/V, the
-positions, optionally the recall head's hidden states) into fixed device
-buffers and replays the graph captured by oda_step_graph_create. The graph
-holds every launch of the step; the Full launches sit behind the IF node the
-gate sets on the device, so no decision travels to the host.
+positions, the gate scores and/or the recall head's hidden states) into fixed
+device buffers and replays the graph captured by oda_step_graph_create. The
+graph holds every launch of the step; the Full launches sit behind the IF
+node the gate sets on the device, so no decision travels to the host.
 
-torch is used for memory and copies only.
+All per-step inputs live in one contiguous "record" (256-byte aligned
+fields), so a step is fed with a single copy, from device or pinned host
+memory. torch is used for memory and copies only.
 """
 
 from __future__ import annotations
@@ -14,6 +16,10 @@ from __future__ import annotations
 from typing import Optional
 
 from . import oda
+
+
+def _align(n: int, a: int = 256) -> int:
+    return (n + a - 1) // a * a
 
 
 class DecodeStep:
@@ -26,14 +32,36 @@ class DecodeStep:
         dt = torch.bfloat16 if c.dtype == oda.BF16 else torch.float32
         dev = "cuda"
         L, hq, hkv, d = c.layers, c.hq, c.hkv, c.head_dim
-        self.q = torch.zeros((L, B, hq, d), dtype=dt, device=dev)
-        self.k_new = torch.zeros((L, B, hkv, d), dtype=dt, device=dev)
-        self.v_new = torch.zeros((L, B, hkv, d), dtype=dt, device=dev)
-        self.seq_lens = torch.ones(B, dtype=torch.int32, device=dev)
+        if recall is None and not external_scores:
+            raise ValueError("without a recall head the gate needs external scores")
+        # ---- input record layout
+        fields = [("q", (L, B, hq, d), dt), ("k_new", (L, B, hkv, d), dt),
+                  ("v_new", (L, B, hkv, d), dt), ("seq_lens", (B,), torch.int32)]
+        if external_scores:
+            fields.append(("gate_scores", (B,), torch.float32))
+        if recall is not None:
+            H = recall["H"]
+            fields += [("h_prev", (B, H), torch.bfloat16), ("emb", (B, H), torch.bfloat16),
+                       ("h_local", (B, H), torch.bfloat16)]
+        self.fields = {}
+        off = 0
+        for name, shape, fdt in fields:
+            n = 1
+            for s in shape:
+                n *= s
+            nbytes = n * torch.empty((), dtype=fdt).element_size()
+            self.fields[name] = (off, shape, fdt, nbytes)
+            off = _align(off + nbytes)
+        self.record_bytes = off
+        self.record = torch.zeros(self.record_bytes, dtype=torch.uint8, device=dev)
+        for name, (o, shape, fdt, nbytes) in self.fields.items():
+            setattr(self, name, self.record[o:o + nbytes].view(fdt).view(shape))
+        if not external_scores:
+            self.gate_scores = None
+        # ---- outputs
         self.out = torch.zeros((L, B, hq, d), dtype=dt, device=dev)
         self.lse = torch.zeros((L, B, hq), dtype=torch.float32, device=dev) if with_lse else None
         self.scores = torch.zeros(B, dtype=torch.float32, device=dev)
-        self.gate_scores = torch.zeros(B, dtype=torch.float32, device=dev) if external_scores else None
         self.flags = torch.zeros(B, dtype=torch.uint8, device=dev)
         self.idx = torch.zeros(B, dtype=torch.int32, device=dev)
         self.count = torch.zeros(1, dtype=torch.int32, device=dev)
@@ -41,15 +69,9 @@ class DecodeStep:
         self.recall = recall
         rk = {}
         if recall is not None:
-            H = recall["H"]
-            self.h_prev = torch.zeros((B, H), dtype=torch.bfloat16, device=dev)
-            self.emb = torch.zeros((B, H), dtype=torch.bfloat16, device=dev)
-            self.h_local = torch.zeros((B, H), dtype=torch.bfloat16, device=dev)
-            rk = dict(h_prev=self.h_prev, emb=self.emb, h_local=self.h_local, H=H,
+            rk = dict(h_prev=self.h_prev, emb=self.emb, h_local=self.h_local, H=recall["H"],
                       W1=recall["W1"], b1=recall["b1"], w2=recall["w2"], b2=recall["b2"],
                       hidden=recall["hidden"])
-        if recall is None and not external_scores:
-            raise ValueError("without a recall head the gate needs external scores")
         self.desc = ctx.step_desc(B=B, q=self.q, k_new=self.k_new, v_new=self.v_new,
                                   seq_lens=self.seq_lens, block_table=block_table,
                                   kv_cache=kv_cache, ring=ring, out=self.out, lse=self.lse,
@@ -57,9 +79,31 @@ class DecodeStep:
                                   flags=self.flags, idx=self.idx, count=self.count, **rk)
         self.graph = ctx.step_graph(self.desc) if graph else None
 
+    # ------------------------------------------------------------- feeding
+    def new_records(self, n: int, device="cuda", pin: bool = False):
+        """Zeroed [n][record_bytes] buffer for pre-packed step records."""
+        import torch
+        r = torch.zeros((n, self.record_bytes), dtype=torch.uint8,
+                        device=device if not pin else "cpu")
+        return r.pin_memory() if pin else r
+
+    def record_view(self, records, i: int, name: str):
+        """View of field `name` inside record i of a records buffer."""
+        o, shape, fdt, nbytes = self.fields[name]
+        return records[i, o:o + nbytes].view(fdt).view(shape)
+
+    def pack(self, records, i: int, **inputs) -> None:
+        for name, val in inputs.items():
+            if val is not None:
+                self.record_view(records, i, name).copy_(val)
+
+    def feed_record(self, records, i: int, non_blocking: bool = True) -> None:
+        """One copy: record i (device or pinned host) -> the static inputs."""
+        self.record.copy_(records[i], non_blocking=non_blocking)
+
     def feed(self, q, k_new, v_new, seq_lens, gate_scores=None, h_prev=None, emb=None,
              h_local=None, non_blocking=True) -> None:
-        """Copy one step's inputs into the static buffers (device or pinned host)."""
+        """Per-field copies into the static inputs (convenience)."""
         self.q.copy_(q, non_blocking=non_blocking)
         self.k_new.copy_(k_new, non_blocking=non_blocking)
         self.v_new.copy_(v_new, non_blocking=non_blocking)

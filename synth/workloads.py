@@ -148,6 +148,19 @@ class Workload:
             q[n.layer, n.row, n.q_head] = self._aim(q[n.layer, n.row, n.q_head], n)
         return q
 
+    def q_step_layer(self, step: int, layer: int) -> np.ndarray:
+        """Storage-dtype queries of one layer for one step, [B][Hq][d], needles applied."""
+        tab = self.q_table()
+        q = np.empty((self.batch, self.hq, self.d), dtype=tab.dtype)
+        for b in range(self.batch):
+            for h in range(self.hq):
+                key = stream_key(self.seed, KIND_Q, layer, b, h)
+                q[b, h] = table_values(key, step * self.d, self.d, tab)
+        for n in self.needles:
+            if n.layer == layer:
+                q[n.row, n.q_head] = self._aim(q[n.row, n.q_head], n)
+        return q
+
     def kv_new_step(self, step: int):
         """(k_new, v_new) for one step, each [L][B][Hkv][d] in storage dtype:
         the history streams at position t0[b] + step."""

@@ -1,0 +1,132 @@
+"""GPU parity at the workloads' full sizes, in the launch configuration the
+benchmark uses (the captured step graph), on outputs the oracle computes one
+(row, layer, KV head) at a time."""
+
+import numpy as np
+import pytest
+
+import oracle as O
+import synth
+from tests import _harness as hx
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def torch():
+    import torch as _t
+    if not _t.cuda.is_available():
+        pytest.skip("needs a GPU")
+    return _t
+
+
+def _check_heads(w, out_step, q_step, step, pairs, flags_row):
+    """out_step: [L][B][hq][d] float64; pairs: (layer, row, kv_head)."""
+    for (l, b, g) in pairs:
+        t = int(w.t0[b]) + step
+        o, _ = hx.oracle_head(w, q_step[l, b], l, b, g, t, full=bool(flags_row[b]))
+        hx.assert_close(out_step[l, b, g * w.group:(g + 1) * w.group], o, *hx.tol(w),
+                        what=f"step {step} layer {l} row {b} head {g}")
+
+
+def test_ctx128k_graph_sampled(torch):
+    """batch 1, 28 layers, t = 131072 + step, Full calls drawn per step:
+    steps 0..6 run through the captured step graph; an unflagged step (1)
+    and two flagged steps (2, 6) are checked on sampled (layer, head) pairs."""
+    from gated_local_full_b200.runtime import DecodeStep
+    w = synth.ctx128k(steps=7)
+    flags = w.flags()[:, 0]
+    assert flags[1] == 0 and flags[2] == 1 and flags[6] == 1
+    ctx, dw = hx.setup(w)
+    st = DecodeStep(ctx, 1, dw.cache, dw.ring, dw.block_table, external_scores=True,
+                    with_lse=True)
+    keep = {}
+    for step in range(w.steps):
+        st.feed(dw.q[step], dw.k_new[step], dw.v_new[step], dw.seq_lens[step],
+                gate_scores=dw.scores[step])
+        st.run()
+        if step in (1, 2, 6):
+            keep[step] = (st.out.to(torch.float64).cpu().numpy(), int(st.count.item()),
+                          st.flags.cpu().numpy().copy())
+    torch.cuda.synchronize()
+    assert ctx.get_device_error() == 0
+    rng = np.random.default_rng(5)
+    for step in (1, 2, 6):
+        out, count, fl = keep[step]
+        assert count == int(flags[step]) and fl[0] == flags[step]
+        q = w.q_step(step)
+        pairs = [(0, 0, 0), (27, 0, 7)] + [(int(rng.integers(1, 27)), 0, int(rng.integers(0, 8)))
+                                           for _ in range(2 if step != 1 else 1)]
+        _check_heads(w, out, q, step, pairs, fl)
+    st.close()
+
+
+@pytest.mark.parametrize("rate", synth.MIXED_RATES)
+def test_mixed_batch(torch, rate):
+    """batch 32, contexts uniform in [4096, 65536], Full calls Bernoulli(rate)
+    per row, append inside the step (graph)."""
+    from gated_local_full_b200.runtime import DecodeStep
+    w = synth.mixed_batch(rate)
+    ctx, dw = hx.setup(w)
+    st = DecodeStep(ctx, w.batch, dw.cache, dw.ring, dw.block_table, external_scores=True)
+    st.feed(dw.q[0], dw.k_new[0], dw.v_new[0], dw.seq_lens[0], gate_scores=dw.scores[0])
+    st.run()
+    torch.cuda.synchronize()
+    assert ctx.get_device_error() == 0
+    flags = w.flags()[0]
+    f, i, c = O.gate(w.scores()[0], 0.0)
+    assert st.flags.cpu().numpy().tolist() == f.tolist() == flags.tolist()
+    assert st.idx.cpu().numpy().tolist() == i.tolist() and int(st.count.item()) == c
+    out = st.out.to(torch.float64).cpu().numpy()
+    q = w.q_step(0)
+    rng = np.random.default_rng(int(rate * 1000))
+    flagged = [b for b in range(w.batch) if flags[b]]
+    # Local for every row (one sampled head each), Full for up to 3 flagged rows
+    pairs = [(0, b, int(rng.integers(0, w.hkv))) for b in range(w.batch) if not flags[b]]
+    pairs += [(0, b, int(rng.integers(0, w.hkv))) for b in flagged[:3]]
+    _check_heads(w, out, q, 0, pairs, flags)
+    st.close()
+
+
+def test_graph_equals_plain_launches_and_skips_full(torch):
+    """The captured step (IF node) and the plain launch sequence give
+    bit-identical outputs; with no flagged row the graph leaves Local."""
+    from gated_local_full_b200.runtime import DecodeStep
+    w = synth.custom("graph", layers=3, batch=4, hq=8, hkv=4, t0=(3000, 100, 2500, 50),
+                     fixed_scores=(1.0, -1.0, 1.0, -1.0), steps=2)
+    res = {}
+    for mode in ("graph", "plain"):
+        ctx, dw = hx.setup(w)
+        st = DecodeStep(ctx, 4, dw.cache, dw.ring, dw.block_table, external_scores=True,
+                        with_lse=True, graph=(mode == "graph"))
+        outs = []
+        for step in range(2):
+            st.feed(dw.q[step], dw.k_new[step], dw.v_new[step], dw.seq_lens[step],
+                    gate_scores=dw.scores[step])
+            st.run()
+            outs.append((st.out.clone(), st.lse.clone()))
+        torch.cuda.synchronize()
+        assert ctx.get_device_error() == 0
+        res[mode] = outs
+        if mode == "graph":
+            # no flagged row: every row must keep its Local output
+            st.feed(dw.q[1], dw.k_new[1], dw.v_new[1], dw.seq_lens[1],
+                    gate_scores=-torch.ones(4, device="cuda"))
+            st.run()
+            torch.cuda.synchronize()
+            assert int(st.count.item()) == 0
+            out = st.out.to(torch.float64).cpu().numpy()
+            q = w.q_step(1)
+            for l in range(3):
+                for b in range(4):
+                    ref = hx.oracle_row(w, 1, l, b)
+                    hx.assert_close(out[l, b], ref["local"], *hx.tol(w), what=f"l{l} b{b}")
+        st.close()
+    for (a, la), (b, lb) in zip(res["graph"], res["plain"]):
+        assert torch.equal(a, b) and torch.equal(la, lb)
+    out = res["graph"][1][0].to(torch.float64).cpu().numpy()
+    for l in range(3):
+        for b in range(4):
+            ref = hx.oracle_row(w, 1, l, b)
+            want = ref["full"] if b % 2 == 0 else ref["local"]
+            hx.assert_close(out[l, b], want, *hx.tol(w), what=f"graph l{l} b{b}")
