@@ -23,6 +23,8 @@
 //   * Warps of a CTA merge their states in shared memory; CTAs sharing a
 //     segment write (m, l, acc) partials and the last one to take the
 //     segment's ticket merges them and writes the output.
+#include <mutex>
+
 #include "oda_internal.cuh"
 
 using namespace oda;
@@ -730,3 +732,141 @@ oda_status launch_attn(oda_ctx* ctx, bool ring_mode, int layer, const void* q,
 }
 
 }  // namespace oda_impl
+
+// ---------------------------------------------------------------------------
+// Full attention without any device allocation.
+//
+// Some callers cannot call cudaMalloc: inference engines that hand the whole
+// GPU to their own pool allocator at start-up (a later cudaMalloc fails once
+// the pool holds the memory, or silently breaks the engine's accounting), and
+// host code on a latency-critical decode loop where a cudaMalloc would
+// synchronize the device. oda_full_attn_gated_static serves them: it needs no
+// context, and the split partials, segment tickets and fallback error word
+// live in the file-scope __device__ arrays below, which every GPU that loads
+// liboda holds until the process exits.
+//
+// In host code these names are host-side stand-ins, not device addresses;
+// the device address of each is fetched once per device with
+// cudaGetSymbolAddress (with that device current) on the first call there.
+// ---------------------------------------------------------------------------
+
+namespace {
+
+constexpr int kStaticPartialFloats = 1 << 18;  // 1 MiB of split partials
+constexpr int kStaticMaxSegments = 512;        // rows x KV heads per call
+constexpr int kStaticMaxCtas = 512;            // persistent grid cap
+constexpr int kStaticMaxDevices = 64;
+
+static __device__ __align__(256) float g_static_partials[kStaticPartialFloats];
+static __device__ __align__(256) int g_static_tickets[kStaticMaxSegments];
+static __device__ __align__(256) int g_static_err[1];
+
+struct StaticDevice {
+  bool ready;
+  float* partials;
+  int* tickets;
+  int* err;
+  int num_sms;
+};
+StaticDevice g_static_dev[kStaticMaxDevices];
+std::mutex g_static_mu;
+
+// Once per device, with that device current: resolve the device addresses.
+oda_status static_setup(int dev, StaticDevice** out) {
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  StaticDevice& s = g_static_dev[dev];
+  if (!s.ready) {
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&s.partials), g_static_partials) !=
+            cudaSuccess ||
+        cudaGetSymbolAddress(reinterpret_cast<void**>(&s.tickets), g_static_tickets) !=
+            cudaSuccess ||
+        cudaGetSymbolAddress(reinterpret_cast<void**>(&s.err), g_static_err) != cudaSuccess ||
+        cudaDeviceGetAttribute(&s.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return ODA_ERR_CUDA;
+    s.ready = true;
+  }
+  *out = &s;
+  return ODA_OK;
+}
+
+struct LaunchStatic {
+  const AttnArgs* a;
+  int num_sms;
+  int max_batch;
+  int B;
+  cudaStream_t st;
+  template <typename T, int D, int G, bool RING>
+  oda_status operator()() {
+    auto k = kernel_ptr<T, D, G, RING>();
+    const size_t sm = smem_bytes<T, D, G, RING>(max_batch);
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) !=
+        cudaSuccess)
+      return ODA_ERR_CUDA;
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, Shape<T, D, G>::W * 32, sm) !=
+            cudaSuccess ||
+        occ < 1)
+      return ODA_ERR_CUDA;
+    int ctas = num_sms * occ;
+    if (ctas > kStaticMaxCtas) ctas = kStaticMaxCtas;
+    // every partial index (CTA + segment) must fit the static array
+    const long long need = (long long)(ctas + B * a->hkv) * G * (D + 2);
+    if (need > kStaticPartialFloats) return ODA_ERR_SHAPE;
+    AttnArgs b = *a;
+    b.min_tiles_per_cta = Shape<T, D, G>::W;
+    b.max_batch = max_batch;
+    k<<<ctas, Shape<T, D, G>::W * 32, sm, st>>>(b);
+    return cudaGetLastError() == cudaSuccess ? ODA_OK : ODA_ERR_CUDA;
+  }
+};
+
+}  // namespace
+
+extern "C" oda_status oda_full_attn_gated_static(const oda_config* cfg, int layer, const void* q,
+                                                 const int32_t* seq_lens,
+                                                 const int32_t* block_table, const void* kv_cache,
+                                                 const int32_t* idx, const int32_t* count,
+                                                 void* out, float* lse, int B, int32_t* err,
+                                                 oda_stream stream) {
+  oda_layout_info lay;
+  const oda_status ls = oda_layout(cfg, &lay);
+  if (ls != ODA_OK) return ls;
+  if (layer < 0 || layer >= cfg->layers || B < 0) return ODA_ERR_ARG;
+  if (B > cfg->max_batch) return ODA_ERR_SHAPE;
+  if (B == 0) return ODA_OK;
+  if (!q || !seq_lens || !block_table || !kv_cache || !idx || !count || !out) return ODA_ERR_ARG;
+  if ((long long)B * cfg->hkv > kStaticMaxSegments) return ODA_ERR_SHAPE;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ODA_ERR_CUDA;
+  if (dev < 0 || dev >= kStaticMaxDevices) return ODA_ERR_SHAPE;
+  StaticDevice* sd = nullptr;
+  oda_status s = static_setup(dev, &sd);
+  if (s != ODA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // tickets must start at zero; a call that gave up early may have left some set
+  if (cudaMemsetAsync(sd->tickets, 0, sizeof(int) * (size_t)B * cfg->hkv, st) != cudaSuccess)
+    return ODA_ERR_CUDA;
+  AttnArgs a;
+  a.q = q;
+  a.out = out;
+  a.lse = lse;
+  a.seq_lens = seq_lens;
+  a.kv = static_cast<const unsigned char*>(kv_cache) +
+         (size_t)layer * (size_t)lay.cache_layer_elems * (size_t)lay.elem_bytes;
+  a.block_table = block_table;
+  a.idx = idx;
+  a.count = count;
+  a.num_blocks = cfg->num_blocks;
+  a.max_blocks = cfg->max_blocks_per_seq;
+  a.B = B;
+  a.hkv = cfg->hkv;
+  a.sink = cfg->sink;
+  a.window = cfg->window;
+  a.ring_blocks = (int)lay.ring_blocks;
+  a.max_batch = cfg->max_batch;
+  a.qscale = 1.4426950408889634f / sqrtf((float)cfg->head_dim);
+  a.partials = sd->partials;
+  a.tickets = sd->tickets;
+  a.err = err ? err : sd->err;
+  return dispatch<false>(*cfg, LaunchStatic{&a, sd->num_sms, cfg->max_batch, B, st});
+}

@@ -31,6 +31,7 @@ EXPORTS = (
     "oda_local_attn", "oda_recall_score", "oda_gate", "oda_full_attn_gated",
     "oda_get_device_error", "oda_selftest_wait_timeout", "oda_step_run",
     "oda_step_graph_create", "oda_step_graph_launch", "oda_step_graph_destroy", "oda_version",
+    "oda_full_attn_gated_static",
 )
 
 
@@ -92,6 +93,8 @@ def lib() -> ctypes.CDLL:
         "oda_step_graph_create": [vp, POINTER(OdaStepDesc), POINTER(c_void_p)],
         "oda_step_graph_launch": [vp, vp],
         "oda_step_graph_destroy": [vp],
+        "oda_full_attn_gated_static": [POINTER(OdaConfig), c_int, vp, vp, vp, vp, vp, vp, vp,
+                                       vp, c_int, vp, vp],
     }
     for name, args in sig.items():
         f = getattr(L, name)
@@ -251,6 +254,17 @@ class OdaContext:
 
     def step_graph(self, desc: OdaStepDesc) -> OdaGraph:
         return OdaGraph(self, desc)
+
+
+def full_attn_gated_static(cfg: OdaConfig, layer, q, seq_lens, block_table, kv_cache, idx,
+                           count, out, lse, B, err=None, stream=None) -> None:
+    """oda_full_attn_gated_static: Full attention with no context and no device
+    allocation (scratch in liboda's fixed device arrays). For callers whose
+    device memory belongs to their own pool allocator."""
+    _check(lib().oda_full_attn_gated_static(ctypes.byref(cfg), layer, ptr(q), ptr(seq_lens),
+                                            ptr(block_table), ptr(kv_cache), ptr(idx),
+                                            ptr(count), ptr(out), ptr(lse), B, ptr(err),
+                                            _stream(stream)), "oda_full_attn_gated_static")
 
 
 def version() -> str:

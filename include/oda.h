@@ -199,6 +199,38 @@ oda_status oda_full_attn_gated(oda_ctx* ctx, int layer, const void* q,
                                const int32_t* count, void* out, float* lse, int B,
                                oda_stream stream);
 
+/*
+ * Full attention for callers that cannot allocate device memory (the pages
+ * have no counterpart; this is an interface for integrators). Engines that
+ * hand the whole GPU to their own pool allocator at start-up cannot have a
+ * library call cudaMalloc later (it fails once the pool holds the memory, or
+ * breaks the pool's accounting), and a cudaMalloc on a latency-critical decode
+ * loop synchronizes the device. This entry point computes exactly what
+ * oda_full_attn_gated computes, with the same arguments, but needs no context
+ * and allocates nothing: its split partials and tickets live in fixed
+ * __device__ arrays inside liboda (1 MiB of partials, 512 segment tickets),
+ * held by every GPU that loads the library until the process exits.
+ *   cfg     host pointer to the model configuration (as for oda_create)
+ *   err     device int32 that receives device-detected errors (ODA_ERR_BOUNDS,
+ *           ODA_ERR_TIMEOUT; first error wins), or NULL to drop them into an
+ *           internal word
+ *   others  as for oda_full_attn_gated
+ * Limits: B * hkv <= 512 segments, and (persistent grid + B * hkv) *
+ * (hq/hkv) * (head_dim + 2) floats within the 1 MiB partials array; larger
+ * calls return ODA_ERR_SHAPE without launching.
+ * The first call on a device resolves the arrays' device addresses
+ * (cudaGetSymbolAddress, with that device current): make that first call
+ * before any stream capture. Every call shares the arrays, which keep the last
+ * call's contents; the tickets are cleared on `stream` before each launch.
+ * Calls that overlap on the GPU (different streams, or another thread's call
+ * in flight) race on the shared arrays and must be serialized by the caller.
+ */
+oda_status oda_full_attn_gated_static(const oda_config* cfg, int layer, const void* q,
+                                      const int32_t* seq_lens, const int32_t* block_table,
+                                      const void* kv_cache, const int32_t* idx,
+                                      const int32_t* count, void* out, float* lse, int B,
+                                      int32_t* err, oda_stream stream);
+
 /* Synchronize `stream`, then return and clear the sticky device error word
  * (ODA_OK if none). Call outside the hot loop. */
 oda_status oda_get_device_error(oda_ctx* ctx, oda_stream stream, int* err);
