@@ -96,9 +96,10 @@ oda_status oda_create(const oda_config* cfg, oda_ctx** out) {
     ctx->max_parts = ctas + cfg->max_batch * cfg->hkv;
     const size_t pbytes = (size_t)ctx->max_parts * g * (cfg->head_dim + 2) * sizeof(float);
     if (cudaMalloc(&ctx->partials, pbytes) != cudaSuccess ||
-        cudaMalloc(&ctx->tickets, (size_t)cfg->max_batch * cfg->hkv * sizeof(int)) != cudaSuccess ||
+        cudaMalloc(&ctx->tickets, 2 * (size_t)cfg->max_batch * cfg->hkv * sizeof(int)) !=
+            cudaSuccess ||
         cudaMalloc(&ctx->err, sizeof(int)) != cudaSuccess ||
-        cudaMemset(ctx->tickets, 0, (size_t)cfg->max_batch * cfg->hkv * sizeof(int)) !=
+        cudaMemset(ctx->tickets, 0, 2 * (size_t)cfg->max_batch * cfg->hkv * sizeof(int)) !=
             cudaSuccess ||
         cudaMemset(ctx->err, 0, sizeof(int)) != cudaSuccess)
       s = ODA_ERR_CUDA;

@@ -29,9 +29,29 @@
 
 using namespace oda;
 
+// Launch shape. The defaults were chosen by measurement on B200; the macros
+// let a build try others without editing the source.
+#ifndef ODA_ATTN_WARPS
+#define ODA_ATTN_WARPS 6
+#endif
+#ifndef ODA_ATTN_STAGES
+#define ODA_ATTN_STAGES 2
+#endif
+#ifndef ODA_RING_TILES_PER_WARP
+#define ODA_RING_TILES_PER_WARP 1
+#endif
+#ifndef ODA_POOL_PERCENT
+#define ODA_POOL_PERCENT 15
+#endif
+#ifndef ODA_FULL_TILES_PER_WARP
+#define ODA_FULL_TILES_PER_WARP 1
+#endif
+
 namespace {
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per barrier wait
+
+
 
 struct AttnArgs {
   const void* q;
@@ -52,51 +72,34 @@ struct AttnArgs {
   int max_batch;
   int min_tiles_per_cta;
   float qscale;                 // log2(e) / sqrt(d)
-  float* partials;
-  int* tickets;
+  float* partials;               // [max_parts][G][d] accumulators, then [max_parts][G][2] (m, l)
+  int max_parts;
+  int* tickets;                 // per segment: CTAs done (reset by the last)
+  int* dyn;                     // per segment: tiles handed out dynamically (reset by the last)
   int* err;
 };
 
+// 16-byte chunk of one K or V row, widened to float pairs (even, odd dims).
 template <typename T>
-struct Vec;
+struct Chunk;
 
-// Loads of DPL consecutive elements of one row, widened to float.
 template <>
-struct Vec<__nv_bfloat16> {
-  template <int DPL>
-  static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&x)[DPL]) {
-    static_assert(DPL == 2 || DPL == 4, "bf16 lanes own 2 or 4 dims");
-    if constexpr (DPL == 4) {
-      const uint2 w = *reinterpret_cast<const uint2*>(p);
-      bf16x2_to_f32(w.x, x[0], x[1]);
-      bf16x2_to_f32(w.y, x[2], x[3]);
-    } else {
-      const uint32_t w = *reinterpret_cast<const uint32_t*>(p);
-      bf16x2_to_f32(w, x[0], x[1]);
-    }
-  }
-  template <int DPL>
-  static __device__ __forceinline__ void store(__nv_bfloat16* p, const float (&x)[DPL]) {
-    for (int i = 0; i < DPL; ++i) p[i] = __float2bfloat16_rn(x[i]);
+struct Chunk<__nv_bfloat16> {
+  static __device__ __forceinline__ void load(const __nv_bfloat16* p, float2 (&x)[4]) {
+    const uint4 w = *reinterpret_cast<const uint4*>(p);
+    bf16x2_to_f32(w.x, x[0].x, x[0].y);
+    bf16x2_to_f32(w.y, x[1].x, x[1].y);
+    bf16x2_to_f32(w.z, x[2].x, x[2].y);
+    bf16x2_to_f32(w.w, x[3].x, x[3].y);
   }
 };
 
 template <>
-struct Vec<float> {
-  template <int DPL>
-  static __device__ __forceinline__ void load(const float* p, float (&x)[DPL]) {
-    static_assert(DPL == 2 || DPL == 4, "f32 lanes own 2 or 4 dims");
-    if constexpr (DPL == 4) {
-      const float4 w = *reinterpret_cast<const float4*>(p);
-      x[0] = w.x; x[1] = w.y; x[2] = w.z; x[3] = w.w;
-    } else {
-      const float2 w = *reinterpret_cast<const float2*>(p);
-      x[0] = w.x; x[1] = w.y;
-    }
-  }
-  template <int DPL>
-  static __device__ __forceinline__ void store(float* p, const float (&x)[DPL]) {
-    for (int i = 0; i < DPL; ++i) p[i] = x[i];
+struct Chunk<float> {
+  static __device__ __forceinline__ void load(const float* p, float2 (&x)[2]) {
+    const float4 w = *reinterpret_cast<const float4*>(p);
+    x[0] = make_float2(w.x, w.y);
+    x[1] = make_float2(w.z, w.w);
   }
 };
 
@@ -148,55 +151,93 @@ __device__ __forceinline__ void normalize(const int* rowstart, int hkv, int hi, 
   }
 }
 
+template <typename T, int D, int G>
+struct Geom {
+  static constexpr int ROWB = D * (int)sizeof(T);   // bytes of one K or V row
+  static constexpr int LPR = ROWB / 16;             // lanes per row (one 16-byte chunk each)
+  static constexpr int DPL = D / LPR;               // dims per lane
+  static constexpr int RPW = 32 / LPR;              // row groups per warp
+  static constexpr int TPL = 16 / RPW;              // tokens per lane per tile
+  static constexpr int V = G * TPL;                 // q.k partial sums per lane per tile
+  static constexpr int NVL = V >= LPR ? V / LPR : 1;  // scores per lane after the reduction
+  static constexpr int DUP = V >= LPR ? 1 : LPR / V;  // lanes holding the same score
+  static constexpr int LPHG = TPL * DUP / NVL;      // lanes of one query head in a row group
+  static constexpr int R = LPR == 8 ? 3 : (LPR == 16 ? 4 : 5);  // butterfly rounds
+  static_assert(LPR == 8 || LPR == 16 || LPR == 32, "row must be 128, 256 or 512 bytes");
+};
+
 template <typename T, int D, int G, int W, int NS, bool RING>
-__global__ void __launch_bounds__(W * 32)
+__global__ void __launch_bounds__(W * 32, 2)
 attn_kernel(const AttnArgs a) {
+  using Gm = Geom<T, D, G>;
   constexpr int TILE_ELEMS = 2 * ODA_TILE * D;
   constexpr int TILE_BYTES = TILE_ELEMS * (int)sizeof(T);
-  constexpr int DPL = D / 32;
-  constexpr int NV16 = 16 * G;                 // partial dot products per lane per tile
-  constexpr int NV = NV16 >= 32 ? NV16 / 32 : 1;   // scores per lane after the butterfly
-  constexpr int DUP = NV16 >= 32 ? 1 : 32 / NV16;  // lanes holding the same score
-  constexpr int LPH = 16 * DUP / NV;           // lanes per query head after the butterfly
+  constexpr int LPR = Gm::LPR, DPL = Gm::DPL, RPW = Gm::RPW, TPL = Gm::TPL;
+  constexpr int V = Gm::V, NVL = Gm::NVL, DUP = Gm::DUP, LPHG = Gm::LPHG;
+  constexpr int DP2 = DPL / 2;                 // float pairs per lane
+  constexpr int PW = G * 16 * 2;               // floats of {p, p} pairs per warp
 
   extern __shared__ __align__(128) unsigned char smem[];
   T* tiles = reinterpret_cast<T*>(smem);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)W * NS * TILE_BYTES);
-  float* pbuf = reinterpret_cast<float*>(bars + W * NS);          // [W][NV16]
-  float* wstate = pbuf + W * NV16;                                 // [W][G][D+2]
-  int* rowstart = reinterpret_cast<int*>(wstate + W * G * (D + 2));  // [max_batch+1]
+  float* wstate = reinterpret_cast<float*>(smem + (size_t)W * NS * TILE_BYTES);  // [W][G][D+2]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(wstate + W * G * (D + 2) + (W * G * (D + 2)) % 2);
+  float* pbuf = reinterpret_cast<float*>(bars + W * NS);          // [W][G][RPW][TPL] x {p,p}
+  int* rowstart = reinterpret_cast<int*>(pbuf + W * PW);          // [max_batch+1]
   int* rowb = rowstart + (a.max_batch + 1);
   int* rowt = rowb + a.max_batch;
-  int* sflag = rowt + a.max_batch;
-  unsigned char* badst = reinterpret_cast<unsigned char*>(sflag + 4);  // [W][NS]
+  int* rowcs = rowt + a.max_batch;                                 // [max_batch+1] CTA prefix
+  int* sflag = rowcs + (a.max_batch + 1);
+  int* sinfo = sflag + 4;                                          // [16] partition of this CTA
+  int* stile = sinfo + 16;                                         // [W][NS] tile of each stage
+  unsigned char* badst = reinterpret_cast<unsigned char*>(stile + W * NS);  // [W][NS]
 
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int warp = tid >> 5;
+  const int rg = lane / LPR;                   // row group: tokens rg, rg+RPW, ...
+  const int li = lane % LPR;                   // 16-byte chunk of the row this lane owns
   const int hq = a.hkv * G;
+  if (tid < W * NS) mbar_init(smem_addr(&bars[tid]), 1);
+  fence_mbar_init();
+  pdl_wait();
+  pdl_launch_dependents();
+  float* pacc = a.partials;                                         // [max_parts][G][D]
+  float* pml = a.partials + (size_t)a.max_parts * G * D;            // [max_parts][G][2]
 
-  // ---------------------------------------------------------------- rows
-  int nrows;
-  if (RING) {
-    nrows = a.B;
-  } else {
-    nrows = *reinterpret_cast<const volatile int32_t*>(a.count);
-    if (nrows < 0 || nrows > a.B) {
-      if (tid == 0 && blockIdx.x == 0) record_error(a.err, ODA_ERR_BOUNDS);
-      nrows = nrows < 0 ? 0 : a.B;
-    }
-  }
-  if (nrows == 0) return;
+  // ------------------------------------------------------- rows, partition
+  // Warp 0 reads the rows, builds the tile prefix and works out this CTA's
+  // share of the tiles (lane-parallel divisions, no block barrier); one
+  // barrier then publishes the result to the other warps through sinfo.
+  //
+  // Partition. "Aligned" when the segments fit the grid: each segment gets
+  // its own CTAs in proportion to its length (at least one, at most one per
+  // min_tiles tiles) and every CTA works inside one segment, so no CTA
+  // finishes one segment's merge before starting the next. Otherwise the
+  // tile space is split evenly and a CTA may span several segments.
   if (warp == 0) {
+    int nr;
+    if (RING) {
+      nr = a.B;
+    } else {
+      nr = *reinterpret_cast<const volatile int32_t*>(a.count);
+      if (nr < 0 || nr > a.B) {
+        if (lane == 0 && blockIdx.x == 0) record_error(a.err, ODA_ERR_BOUNDS);
+        nr = nr < 0 ? 0 : a.B;
+      }
+    }
     int carry = 0;
-    for (int base = 0; base < nrows; base += 32) {
+    for (int base = 0; base < nr; base += 32) {
       const int i = base + lane;
       int nt = 0;
-      if (i < nrows) {
-        const int b = RING ? i : a.idx[i];
-        const bool okb = b >= 0 && b < a.B;
-        const int t = okb ? a.seq_lens[b] : 0;
-        if (!okb || t < 1) {
+      // with B <= 32 every lane loads one row's length alongside the index,
+      // so the two loads overlap instead of chaining (all lanes shuffle)
+      const int tl = (a.B <= 32 && lane < a.B) ? a.seq_lens[lane] : 0;
+      const int bl = i < nr ? (RING ? i : a.idx[i]) : 0;
+      const bool okl = bl >= 0 && bl < a.B;
+      const int ts = __shfl_sync(0xffffffffu, tl, okl ? (bl & 31) : 0);
+      if (i < nr) {
+        const int t = !okl ? 0 : (a.B <= 32 ? ts : a.seq_lens[bl]);
+        if (!okl || t < 1) {
           if (blockIdx.x == 0) record_error(a.err, ODA_ERR_BOUNDS);
         } else if (RING) {
           nt = (a.sink + min(t, a.window) + ODA_TILE - 1) / ODA_TILE;
@@ -207,7 +248,7 @@ attn_kernel(const AttnArgs a) {
             nt = 0;
           }
         }
-        rowb[i] = okb ? b : 0;
+        rowb[i] = okl ? bl : 0;
         rowt[i] = t;
       }
       int v = nt * a.hkv;
@@ -216,60 +257,181 @@ attn_kernel(const AttnArgs a) {
         int y = __shfl_up_sync(0xffffffffu, v, o);
         if (lane >= o) v += y;
       }
-      if (i < nrows) rowstart[i + 1] = carry + v;
+      if (i < nr) rowstart[i + 1] = carry + v;
       carry += __shfl_sync(0xffffffffu, v, 31);
     }
-    if (lane == 0) rowstart[0] = 0;
+    __syncwarp();                               // rowstart[] visible to every lane
+    const int tot = carry;
+    int P = (int)gridDim.x;
+    if (tot > 0) P = min(P, max(1, (tot + a.min_tiles_per_cta - 1) / a.min_tiles_per_cta));
+    // per-row CTA counts of the aligned partition, their prefix, the worst load
+    int carry2 = 0, worst = 0;
+    for (int base = 0; base < nr; base += 32) {
+      const int i = base + lane;
+      int n = 0;
+      if (i < nr) {
+        const int nt = (rowstart[i + 1] - (i == 0 ? 0 : rowstart[i])) / a.hkv;
+        if (nt > 0) {
+          n = ((unsigned)nt < (1u << 31) / (unsigned)P)
+                  ? (int)(((unsigned)nt * (unsigned)P) / (unsigned)tot)
+                  : (int)(((long long)nt * P) / tot);
+          n = max(min(n, nt / a.min_tiles_per_cta), 1);
+          worst = max(worst, (nt + n - 1) / n);
+        }
+      }
+      int v = n * a.hkv;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        int y = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += y;
+      }
+      if (i < nr) rowcs[i + 1] = carry2 + v;
+      carry2 += __shfl_sync(0xffffffffu, v, 31);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) worst = max(worst, __shfl_xor_sync(0xffffffffu, worst, o));
+    __syncwarp();
+    if (lane == 0) {
+      rowstart[0] = 0;
+      rowcs[0] = 0;
+      const int cta0 = (int)blockIdx.x;
+      // aligned only if it fits the grid and no CTA gets more than 1.2x the
+      // even share of tiles
+      const int even = tot > 0 ? (tot + P - 1) / P : 0;
+      const bool al = tot > 0 && carry2 <= (int)gridDim.x && 5 * worst <= 6 * even;
+      int lo_ = 0, hi_ = 0, pb = 0, np = 0, pa = 0, vc = cta0;
+      if (tot > 0 && al && cta0 < carry2) {
+        vc = cta0;
+        int r0 = 0, r1 = nr - 1;                     // row with rowcs[r0] <= vc < rowcs[r0+1]
+        while (r0 < r1) {
+          const int mid = (r0 + r1 + 1) >> 1;
+          if (rowcs[mid] <= vc) r0 = mid; else r1 = mid - 1;
+        }
+        const int nt = (rowstart[r0 + 1] - rowstart[r0]) / a.hkv;
+        const int n = (rowcs[r0 + 1] - rowcs[r0]) / a.hkv;
+        const int g = (vc - rowcs[r0]) / n, part = vc - rowcs[r0] - g * n;
+        const int s0a = rowstart[r0] + g * nt;
+        if ((unsigned)nt < (1u << 31) / (unsigned)(n + 1)) {
+          lo_ = s0a + (int)(((unsigned)part * (unsigned)nt) / (unsigned)n);
+          hi_ = s0a + (int)(((unsigned)(part + 1) * (unsigned)nt) / (unsigned)n);
+        } else {
+          lo_ = s0a + (int)(((long long)part * nt) / n);
+          hi_ = s0a + (int)(((long long)(part + 1) * nt) / n);
+        }
+        pb = rowcs[r0] + g * n;
+        np = n;
+        pa = part;
+      } else if (tot > 0 && !al && cta0 < P) {
+        lo_ = (int)(((long long)cta0 * tot) / P);
+        hi_ = (int)(((long long)(cta0 + 1) * tot) / P);
+      }
+      sinfo[0] = nr; sinfo[1] = tot; sinfo[2] = P; sinfo[3] = al ? 1 : 0;
+      sinfo[4] = lo_; sinfo[5] = hi_; sinfo[6] = pb; sinfo[7] = np; sinfo[8] = pa;
+      sinfo[9] = vc;
+    }
   }
   __syncthreads();
-  const int total = rowstart[nrows];
-  if (total == 0) return;
-  int P = (int)gridDim.x;
-  {
-    const int want = max(1, (total + a.min_tiles_per_cta - 1) / a.min_tiles_per_cta);
-    P = min(P, want);
-  }
+  const int nrows = sinfo[0];
+  const int total = sinfo[1];
+  const int P = sinfo[2];
+  const bool aligned = sinfo[3] != 0;
+  int lo = sinfo[4], hi = sinfo[5];
+  const int pbase_al = sinfo[6], nparts_al = sinfo[7], part_al = sinfo[8], vcta = sinfo[9];
   const int cta = (int)blockIdx.x;
-  if (cta >= P) return;
-  const int lo = (int)(((long long)cta * total) / P);
-  const int hi = (int)(((long long)(cta + 1) * total) / P);
-  if (lo >= hi) return;
+  if (nrows == 0 || total == 0 || lo >= hi) return;
 
-  if (tid < W * NS) mbar_init(smem_addr(&bars[tid]), 1);
-  fence_mbar_init();
-  __syncthreads();
-
-  const uint64_t policy = RING ? l2_policy_evict_last() : l2_policy_evict_first();
+  // K/V is read once per launch: stream it through L2 (the ring too, so no
+  // layer's window stays resident from one step to the next)
+  const uint64_t policy = l2_policy_evict_first();
   const T* kvbase = reinterpret_cast<const T*>(a.kv);
 
   // -------------------------------------------------------- tile producer
+  // Each warp walks its CTA's tile range with stride W. In the aligned
+  // partition a long segment keeps its last ODA_POOL_PERCENT % of tiles in a
+  // pool: a warp that finishes its static share takes pool tiles one at a
+  // time from the segment's counter (two grabs kept in flight), so warps
+  // that stream faster take more and the segment's CTAs finish together.
   Cursor prod;
   prod.k = lo;
   locate(rowstart, nrows, a.hkv, lo, prod);
+  const int seg_b = rowb[prod.i];
+  const int seg_nt = prod.nt;
+  const int seg_s0 = prod.s1 - prod.nt;
+  const int sigma0 = prod.i * a.hkv + prod.g;
+  int pool0 = seg_nt;                        // first pool tile (relative); == nt: no pool
+  if (aligned && seg_nt >= 8 * nparts_al * W) {
+    pool0 = seg_nt - max(2 * nparts_al * W, seg_nt * ODA_POOL_PERCENT / 100);
+    // static share of this CTA within [0, pool0)
+    lo = seg_s0 + (int)(((long long)part_al * pool0) / nparts_al);
+    hi = seg_s0 + (int)(((long long)(part_al + 1) * pool0) / nparts_al);
+  }
+  const bool use_pool = pool0 < seg_nt;
+  int q0 = seg_nt, q1 = seg_nt, qb0 = -1, qb1 = -1;   // lane 0: grabbed pool tiles, blocks
+  auto grab = [&](int& q, int& qb) {                  // lane 0 only
+    q = pool0 + atomicAdd(&a.dyn[sigma0], 1);
+    qb = (!RING && q < seg_nt) ? a.block_table[(long long)seg_b * a.max_blocks + q] : -1;
+  };
   prod.k = lo + warp;
+  if (prod.k >= hi) prod.k = hi;
   normalize(rowstart, a.hkv, hi, warp, prod);
-  Cursor cons = prod;
 
-  auto issue = [&](const Cursor& c, int stage) {
+  // Block ids of the producer's next 32 tiles of the current row, one per
+  // lane, so the per-tile issue does not wait on a global load.
+  int bc_row = -1, bc_base = 0, bc_val = -1;
+
+  // Warp-uniform: the next tile of this warp. Returns false when done.
+  // Sets (k, i, g, nt, blk); blk < -1 means "look it up in the block cache".
+  auto next_tile = [&](int& k, int& i, int& g, int& nt, int& blk) -> bool {
+    if (prod.k < hi) {
+      k = prod.k; i = prod.i; g = prod.g; nt = prod.nt; blk = -2;
+      prod.k += W;
+      normalize(rowstart, a.hkv, hi, warp, prod);
+      return true;
+    }
+    if (!use_pool) return false;
+    const int rel = __shfl_sync(0xffffffffu, q0, 0);
+    blk = __shfl_sync(0xffffffffu, qb0, 0);
+    if (rel >= seg_nt) return false;
+    if (lane == 0) {
+      q0 = q1;
+      qb0 = qb1;
+      grab(q1, qb1);
+    }
+    k = seg_s0 + rel; i = prod.i; g = prod.g; nt = seg_nt;
+    return true;
+  };
+
+  // Warp-uniform; lane 0 issues the copy and records the stage's tile.
+  auto issue = [&](int k, int i, int g, int nt, int blk_in, int stage) {
+    const int b = rowb[i];
+    const int jt = k - (rowstart[i] + g * nt);
+    const T* src;
+    bool bad = false;
+    if (RING) {
+      src = kvbase + (((long long)b * a.hkv + g) * a.ring_blocks + jt) * TILE_ELEMS;
+    } else {
+      int blk = blk_in;
+      if (blk < -1) {
+        if (i != bc_row || jt < bc_base || jt >= bc_base + 32 * W || (jt - bc_base) % W != 0) {
+          bc_row = i;
+          bc_base = jt;
+          const int jl = jt + lane * W;
+          bc_val = jl < nt ? a.block_table[(long long)b * a.max_blocks + jl] : -1;
+        }
+        blk = __shfl_sync(0xffffffffu, bc_val, (jt - bc_base) / W);
+      }
+      bad = blk < 0 || (long long)blk >= a.num_blocks;
+      src = kvbase + ((long long)blk * a.hkv + g) * TILE_ELEMS;
+    }
     if (lane == 0) {
       const uint32_t bar = smem_addr(&bars[warp * NS + stage]);
-      const uint32_t dst = smem_addr(tiles + (size_t)(warp * NS + stage) * TILE_ELEMS);
-      const int b = rowb[c.i];
-      const int jt = c.k - (c.s1 - c.nt);
-      const T* src;
-      bool bad = false;
-      if (RING) {
-        src = kvbase + (((long long)b * a.hkv + c.g) * a.ring_blocks + jt) * TILE_ELEMS;
-      } else {
-        const int blk = a.block_table[(long long)b * a.max_blocks + jt];
-        bad = blk < 0 || (long long)blk >= a.num_blocks;
-        src = kvbase + ((long long)blk * a.hkv + c.g) * TILE_ELEMS;
-      }
+      stile[warp * NS + stage] = k;
       badst[warp * NS + stage] = bad ? 1 : 0;
       if (bad) {
         record_error(a.err, ODA_ERR_BOUNDS);
         mbar_arrive(bar);
       } else {
+        const uint32_t dst = smem_addr(tiles + (size_t)(warp * NS + stage) * TILE_ELEMS);
         mbar_arrive_expect_tx(bar, TILE_BYTES);
         bulk_g2s(dst, src, TILE_BYTES, bar, policy);
       }
@@ -277,14 +439,19 @@ attn_kernel(const AttnArgs a) {
   };
 
   int issued = 0;
+  bool prod_done = false;
 #pragma unroll 1
-  for (int s = 0; s < NS; ++s) {
-    if (prod.k >= hi) break;
-    issue(prod, s);
+  for (int st2 = 0; st2 < NS; ++st2) {
+    int k, i, g, nt, blk;
+    if (!next_tile(k, i, g, nt, blk)) { prod_done = true; break; }
+    issue(k, i, g, nt, blk, st2);
     ++issued;
-    prod.k += W;
-    normalize(rowstart, a.hkv, hi, warp, prod);
   }
+  if (use_pool && lane == 0) {       // after the first copies are in flight
+    grab(q0, qb0);
+    grab(q1, qb1);
+  }
+  __syncwarp();
   int consumed = 0;
   int waited = 0;        // tiles whose copy is known to have landed
   bool aborted = false;
@@ -298,23 +465,22 @@ attn_kernel(const AttnArgs a) {
     const int t = rowt[seg.i];
     const int s0 = seg.s1 - seg.nt;
 
-    float qv[G][DPL];
+    // this lane's DPL dims of the G query heads (exact, unscaled)
+    float2 q2[G][DP2];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       const T* qp = reinterpret_cast<const T*>(a.q) +
-                    ((long long)b * hq + seg.g * G + h) * D + lane * DPL;
-      float x[DPL];
-      Vec<T>::template load<DPL>(qp, x);
-#pragma unroll
-      for (int e = 0; e < DPL; ++e) qv[h][e] = x[e] * a.qscale;
+                    ((long long)b * hq + seg.g * G + h) * D + li * DPL;
+      Chunk<T>::load(qp, q2[h]);
     }
-    float m_run[G], l_run[G], acc[G][DPL];
+    float m_run[G], l_run[G];
+    float2 acc[G][DP2];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       m_run[h] = -INFINITY;
       l_run[h] = 0.f;
 #pragma unroll
-      for (int e = 0; e < DPL; ++e) acc[h][e] = 0.f;
+      for (int e = 0; e < DP2; ++e) acc[h][e] = make_float2(0.f, 0.f);
     }
 
     // ring validity constants of this row
@@ -322,8 +488,10 @@ attn_kernel(const AttnArgs a) {
     const int nsv = min(max(t - a.window, 0), a.sink);
 
 #pragma unroll 1
-    while (cons.k < hi && cons.i == seg.i && cons.g == seg.g) {
+    while (consumed < issued) {
       const int stage = consumed % NS;
+      const int ktile = stile[warp * NS + stage];
+      if (ktile >= seg.s1) break;              // the next tile belongs to a later segment
       const uint32_t parity = (uint32_t)((consumed / NS) & 1);
       if (!aborted) {
         // every lane waits; the warp proceeds only if all of them saw the data
@@ -336,7 +504,7 @@ attn_kernel(const AttnArgs a) {
           if (lane == 0) record_error(a.err, ODA_ERR_TIMEOUT);
         }
       }
-      const int jt = cons.k - s0;
+      const int jt = ktile - s0;
       uint32_t mask;
       if (RING) {
         const int base = jt * ODA_TILE;
@@ -350,31 +518,31 @@ attn_kernel(const AttnArgs a) {
       if (mask) {
         const T* tk = tiles + (size_t)(warp * NS + stage) * TILE_ELEMS;
         const T* tv = tk + ODA_TILE * D;
-        // ---- q.k partial sums: x[h*16 + j]
-        float x[NV16];
+        // ---- q.k partial sums over this lane's chunk: x[h*TPL + u], token rg + RPW*u
+        float x[V];
 #pragma unroll
-        for (int j = 0; j < ODA_TILE; ++j) {
-          float kf[DPL];
-          Vec<T>::template load<DPL>(tk + j * D + lane * DPL, kf);
+        for (int u = 0; u < TPL; ++u) {
+          float2 kf[DP2];
+          Chunk<T>::load(tk + (rg + RPW * u) * D + li * DPL, kf);
 #pragma unroll
           for (int h = 0; h < G; ++h) {
-            float s = 0.f;
+            float2 s2 = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int e = 0; e < DPL; ++e) s = fmaf(qv[h][e], kf[e], s);
-            x[h * 16 + j] = s;
+            for (int e = 0; e < DP2; ++e) s2 = __ffma2_rn(q2[h][e], kf[e], s2);
+            x[h * TPL + u] = s2.x + s2.y;
           }
         }
-        // ---- transposing butterfly: lane ends with full sums of its slots
+        // ---- transposing butterfly over the LPR lanes of the row group
         {
-          int c = NV16;
+          int c = V;
 #pragma unroll
-          for (int r = 0; r < 5; ++r) {
-            const int off = 16 >> r;
+          for (int r = 0; r < Gm::R; ++r) {
+            const int off = LPR >> (r + 1);
             if (c > 1) {
               const bool upper = (lane & off) != 0;
               const int half = c >> 1;
 #pragma unroll
-              for (int i2 = 0; i2 < NV16 / 2; ++i2) {
+              for (int i2 = 0; i2 < V / 2; ++i2) {
                 if (i2 < half) {
                   const float send = upper ? x[i2] : x[i2 + half];
                   const float keep = upper ? x[i2 + half] : x[i2];
@@ -387,110 +555,130 @@ attn_kernel(const AttnArgs a) {
             }
           }
         }
-        // slot index of x[e] on this lane
-        float sc[NV];
-        int myh;
+        // scores of this lane: index v = h*TPL + u, token rg + RPW*u
+        float sc[NVL];
+        int myh = 0;
 #pragma unroll
-        for (int e = 0; e < NV; ++e) {
-          const int v = NV16 >= 32 ? lane * NV + e : lane / DUP;
-          const int j = v & 15;
-          myh = v >> 4;
-          sc[e] = ((mask >> j) & 1u) ? x[e] : -INFINITY;
+        for (int e = 0; e < NVL; ++e) {
+          const int v = V >= LPR ? li * NVL + e : li / DUP;
+          const int u = v % TPL;
+          myh = v / TPL;
+          const int j = rg + RPW * u;
+          sc[e] = ((mask >> j) & 1u) ? x[e] * a.qscale : -INFINITY;
         }
-        // ---- per-head tile max
+        // ---- per-head tile max (within the row group, then across groups)
         float mx = sc[0];
 #pragma unroll
-        for (int e = 1; e < NV; ++e) mx = fmaxf(mx, sc[e]);
+        for (int e = 1; e < NVL; ++e) mx = fmaxf(mx, sc[e]);
 #pragma unroll
-        for (int o = DUP; o < LPH; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        for (int o = DUP; o < LPHG; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+#pragma unroll
+        for (int o = LPR; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
         float m_new[G], alpha[G];
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-          const float th = __shfl_sync(0xffffffffu, mx, h * LPH);
+          const float th = __shfl_sync(0xffffffffu, mx, h * LPHG);
           m_new[h] = fmaxf(m_run[h], th);
           alpha[h] = (m_run[h] == -INFINITY) ? 0.f : fast_exp2(m_run[h] - m_new[h]);
         }
         float mine = m_new[0];
 #pragma unroll
         for (int h = 1; h < G; ++h) if (myh == h) mine = m_new[h];
-        float p[NV];
+        float p[NVL];
         float ps = 0.f;
 #pragma unroll
-        for (int e = 0; e < NV; ++e) {
+        for (int e = 0; e < NVL; ++e) {
           p[e] = (sc[e] == -INFINITY) ? 0.f : fast_exp2(sc[e] - mine);
           ps += p[e];
         }
 #pragma unroll
-        for (int o = DUP; o < LPH; o <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
+        for (int o = DUP; o < LPHG; o <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
+#pragma unroll
+        for (int o = LPR; o < 32; o <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-          const float tsum = __shfl_sync(0xffffffffu, ps, h * LPH);
+          const float tsum = __shfl_sync(0xffffffffu, ps, h * LPHG);
           l_run[h] = l_run[h] * alpha[h] + tsum;
           m_run[h] = m_new[h];
+          const float2 a2 = make_float2(alpha[h], alpha[h]);
 #pragma unroll
-          for (int e = 0; e < DPL; ++e) acc[h][e] *= alpha[h];
+          for (int e = 0; e < DP2; ++e) acc[h][e] = __fmul2_rn(acc[h][e], a2);
         }
-        // ---- probabilities to shared memory, then P.V
-        float* pw = pbuf + warp * NV16;
+        // ---- {p, p} pairs to shared memory, laid out [G][RPW][TPL]
+        float2* pw = reinterpret_cast<float2*>(pbuf + warp * PW);
+        if (li % DUP == 0) {
 #pragma unroll
-        for (int e = 0; e < NV; ++e) {
-          const int v = NV16 >= 32 ? lane * NV + e : lane / DUP;
-          if (NV16 >= 32 || (lane % DUP) == 0) pw[v] = p[e];
+          for (int e = 0; e < NVL; ++e) {
+            const int v = V >= LPR ? li * NVL + e : li / DUP;
+            pw[((v / TPL) * RPW + rg) * TPL + v % TPL] = make_float2(p[e], p[e]);
+          }
         }
         __syncwarp();
+        // ---- P.V over this row group's tokens
         if (mask == 0xFFFFu) {
 #pragma unroll
-          for (int j4 = 0; j4 < ODA_TILE; j4 += 4) {
-            float4 pj[G];
+          for (int u = 0; u < TPL; ++u) {
+            float2 vf[DP2];
+            Chunk<T>::load(tv + (rg + RPW * u) * D + li * DPL, vf);
 #pragma unroll
-            for (int h = 0; h < G; ++h) pj[h] = *reinterpret_cast<const float4*>(pw + h * 16 + j4);
+            for (int h = 0; h < G; ++h) {
+              const float2 pp = pw[(h * RPW + rg) * TPL + u];
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-              float vf[DPL];
-              Vec<T>::template load<DPL>(tv + (j4 + jj) * D + lane * DPL, vf);
-#pragma unroll
-              for (int h = 0; h < G; ++h) {
-                const float pp = jj == 0 ? pj[h].x : jj == 1 ? pj[h].y : jj == 2 ? pj[h].z : pj[h].w;
-#pragma unroll
-                for (int e = 0; e < DPL; ++e) acc[h][e] = fmaf(pp, vf[e], acc[h][e]);
-              }
+              for (int e = 0; e < DP2; ++e) acc[h][e] = __ffma2_rn(pp, vf[e], acc[h][e]);
             }
           }
         } else {
 #pragma unroll 1
-          for (int j = 0; j < ODA_TILE; ++j) {
-            if (!((mask >> j) & 1u)) continue;   // masked slots may hold garbage
-            float vf[DPL];
-            Vec<T>::template load<DPL>(tv + j * D + lane * DPL, vf);
+          for (int u = 0; u < TPL; ++u) {
+            if (!((mask >> (rg + RPW * u)) & 1u)) continue;   // masked slots may hold garbage
+            float2 vf[DP2];
+            Chunk<T>::load(tv + (rg + RPW * u) * D + li * DPL, vf);
 #pragma unroll
             for (int h = 0; h < G; ++h) {
-              const float pp = pw[h * 16 + j];
+              const float2 pp = pw[(h * RPW + rg) * TPL + u];
 #pragma unroll
-              for (int e = 0; e < DPL; ++e) acc[h][e] = fmaf(pp, vf[e], acc[h][e]);
+              for (int e = 0; e < DP2; ++e) acc[h][e] = __ffma2_rn(pp, vf[e], acc[h][e]);
             }
           }
         }
       }
       __syncwarp();
       // refill the stage just consumed
-      if (prod.k < hi && !aborted) {
-        issue(prod, stage);
-        ++issued;
-        prod.k += W;
-        normalize(rowstart, a.hkv, hi, warp, prod);
+      if (!prod_done && !aborted) {
+        int k, i, g, nt, blk;
+        if (next_tile(k, i, g, nt, blk)) {
+          issue(k, i, g, nt, blk, stage);
+          ++issued;
+        } else {
+          prod_done = true;
+        }
+        __syncwarp();
       }
       ++consumed;
-      cons.k += W;
-      normalize(rowstart, a.hkv, hi, warp, cons);
     }
 
     // ---------------------------------------------- merge warps of the CTA
+    // row groups hold disjoint tokens under the same running max: add them
+#pragma unroll
+    for (int o = LPR; o < 32; o <<= 1)
+#pragma unroll
+      for (int h = 0; h < G; ++h)
+#pragma unroll
+        for (int e = 0; e < DP2; ++e) {
+          acc[h][e].x += __shfl_xor_sync(0xffffffffu, acc[h][e].x, o);
+          acc[h][e].y += __shfl_xor_sync(0xffffffffu, acc[h][e].y, o);
+        }
     float* ws = wstate + (size_t)warp * G * (D + 2);
+    if (rg == 0) {
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
+      for (int h = 0; h < G; ++h)
 #pragma unroll
-      for (int e = 0; e < DPL; ++e) ws[h * (D + 2) + lane * DPL + e] = acc[h][e];
-      if (lane == 0) {
+        for (int e = 0; e < DP2; ++e)
+          *reinterpret_cast<float2*>(ws + h * (D + 2) + li * DPL + 2 * e) = acc[h][e];
+    }
+    if (lane == 0) {
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
         ws[h * (D + 2) + D] = m_run[h];
         ws[h * (D + 2) + D + 1] = l_run[h];
       }
@@ -498,10 +686,20 @@ attn_kernel(const AttnArgs a) {
     __syncthreads();
 
     const int sigma = seg.i * a.hkv + seg.g;
-    const long long Pll = P;
-    const int c_first = (int)(((long long)(s0 + 1) * Pll - 1) / total);
-    const int c_last = (int)(((long long)seg.s1 * Pll - 1) / total);
-    const int nparts = c_last - c_first + 1;
+    // the segment's partials are pbase .. pbase+nparts-1; this CTA writes mypart
+    int pbase, nparts, mypart;
+    if (aligned) {
+      pbase = pbase_al;
+      nparts = nparts_al;
+      mypart = vcta;
+    } else {
+      const long long Pll = P;
+      const int c_first = (int)(((long long)(s0 + 1) * Pll - 1) / total);
+      const int c_last = (int)(((long long)seg.s1 * Pll - 1) / total);
+      pbase = c_first + sigma;
+      nparts = c_last - c_first + 1;
+      mypart = cta + sigma;
+    }
     const int hglob0 = seg.g * G;
     T* outp = reinterpret_cast<T*>(a.out);
 
@@ -526,9 +724,9 @@ attn_kernel(const AttnArgs a) {
           a.lse[(long long)b * hq + hglob0 + h] =
               lt > 0.f ? (mt + fast_log2(lt)) * 0.69314718055994531f : -INFINITY;
       } else {
-        float* pp = a.partials + ((long long)(cta + sigma) * G + h) * (D + 2);
-        pp[dd] = at;
-        if (dd == 0) { pp[D] = mt; pp[D + 1] = lt; }
+        const long long pidx = (long long)mypart * G + h;
+        pacc[pidx * D + dd] = at;
+        if (dd == 0) { pml[pidx * 2] = mt; pml[pidx * 2 + 1] = lt; }
       }
     }
     if (nparts > 1) {
@@ -541,30 +739,135 @@ attn_kernel(const AttnArgs a) {
       __syncthreads();
       if (sflag[0]) {
         __threadfence();
-        for (int o = tid; o < G * D; o += W * 32) {
-          const int h = o / D, dd = o % D;
-          float mt = -INFINITY;
-          for (int c2 = c_first; c2 <= c_last; ++c2)
-            mt = fmaxf(mt, __ldcg(a.partials + ((long long)(c2 + sigma) * G + h) * (D + 2) + D));
-          float lt = 0.f, at = 0.f;
-          if (mt != -INFINITY) {
-            for (int c2 = c_first; c2 <= c_last; ++c2) {
-              const float* pp = a.partials + ((long long)(c2 + sigma) * G + h) * (D + 2);
-              const float pm = __ldcg(pp + D);
-              if (pm == -INFINITY) continue;
-              const float sc2 = fast_exp2(pm - mt);
-              lt += __ldcg(pp + D + 1) * sc2;
-              at += __ldcg(pp + dd) * sc2;
+        // Last CTA of the segment: merge its nparts partials. The accumulator
+        // loads are issued before the (m, l) reduction so both travel in one
+        // L2 round trip.
+        constexpr int NCH = G * D / 4;                 // float4 chunks of the output
+        constexpr int SPLIT = (W * 32) / NCH > 0 ? (W * 32) / NCH : 1;
+        constexpr int MAXB = G >= 4 ? 4 : 8;           // partial chunks held per thread
+        float* sml = wstate;                           // [nparts][G][2]
+        float* ssc = sml + 2 * nparts * G;             // [nparts][G] scale factors
+        float* stot = ssc + nparts * G;                // [2G]: m_tot, l_tot
+        const int comb_off = (3 * nparts * G + 2 * G + 3) & ~3;
+        float4* scomb = reinterpret_cast<float4*>(wstate + comb_off);   // [SPLIT-1][NCH]
+        const bool fits = comb_off + 4 * NCH * (SPLIT - 1) <= W * G * (D + 2) &&
+                          (SPLIT > 1 || NCH <= W * 32) && nparts <= SPLIT * MAXB * 4;
+        if (!fits) {
+          // many partials (few segments over a large grid): one output element
+          // per thread, partials in turn
+          for (int o = tid; o < G * D; o += W * 32) {
+            const int h = o / D, dd = o % D;
+            float mt = -INFINITY;
+            for (int j = 0; j < nparts; ++j)
+              mt = fmaxf(mt, __ldcg(pml + ((long long)(pbase + j) * G + h) * 2));
+            float lt = 0.f, at = 0.f;
+            if (mt != -INFINITY) {
+              for (int j = 0; j < nparts; ++j) {
+                const long long pidx = (long long)(pbase + j) * G + h;
+                const float pm = __ldcg(pml + pidx * 2);
+                if (pm == -INFINITY) continue;
+                const float sc2 = fast_exp2(pm - mt);
+                lt += __ldcg(pml + pidx * 2 + 1) * sc2;
+                at += __ldcg(pacc + pidx * D + dd) * sc2;
+              }
+            }
+            const long long orow = ((long long)b * hq + hglob0 + h) * D;
+            outp[orow + dd] = (T)(lt > 0.f ? at / lt : 0.f);
+            if (dd == 0 && a.lse)
+              a.lse[(long long)b * hq + hglob0 + h] =
+                  lt > 0.f ? (mt + fast_log2(lt)) * 0.69314718055994531f : -INFINITY;
+          }
+        } else {
+          // thread -> (output chunk ch, partials part, part + SPLIT, ...)
+          const int ch = tid % NCH;
+          const int part = (tid / NCH < SPLIT && tid < NCH * SPLIT) ? tid / NCH : SPLIT;
+          const int hch = (ch * 4) / D;
+          float4 s4 = make_float4(0.f, 0.f, 0.f, 0.f);
+          float4 v4[MAXB];
+          int nb = 0;                                   // chunks loaded in the first batch
+          if (part < SPLIT) {
+#pragma unroll
+            for (int u = 0; u < MAXB; ++u) {
+              const int j = part + u * SPLIT;
+              if (j < nparts) {
+                v4[u] = __ldcg(reinterpret_cast<const float4*>(
+                    pacc + (long long)(pbase + j) * G * D) + ch);
+                nb = u + 1;
+              }
             }
           }
-          const long long orow = ((long long)b * hq + hglob0 + h) * D;
-          outp[orow + dd] = (T)(lt > 0.f ? at / lt : 0.f);
-          if (dd == 0 && a.lse)
-            a.lse[(long long)b * hq + hglob0 + h] =
-                lt > 0.f ? (mt + fast_log2(lt)) * 0.69314718055994531f : -INFINITY;
+          // (a) every partial's (m, l)
+          for (int i = tid; i < nparts * G; i += W * 32) {
+            const float2 ml = __ldcg(reinterpret_cast<const float2*>(
+                pml + ((long long)(pbase + i / G) * G + (i % G)) * 2));
+            sml[2 * i] = ml.x;
+            sml[2 * i + 1] = ml.y;
+          }
+          __syncthreads();
+          // (b) one warp per head: max, per-partial scales, normaliser
+          if (warp < G) {
+            const int h = warp;
+            float mx = -INFINITY;
+            for (int j = lane; j < nparts; j += 32) mx = fmaxf(mx, sml[2 * (j * G + h)]);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            float ls = 0.f;
+            for (int j = lane; j < nparts; j += 32) {
+              const float pm = sml[2 * (j * G + h)];
+              const float s2 = (pm == -INFINITY || mx == -INFINITY) ? 0.f : fast_exp2(pm - mx);
+              ssc[j * G + h] = s2;
+              ls += sml[2 * (j * G + h) + 1] * s2;
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
+            if (lane == 0) { stot[h] = mx; stot[G + h] = ls; }
+          }
+          __syncthreads();
+          // (c) weighted sums of the held chunks, then any remaining batches
+          if (part < SPLIT) {
+#pragma unroll
+            for (int u = 0; u < MAXB; ++u) {
+              if (u < nb) {
+                const float w4 = ssc[(part + u * SPLIT) * G + hch];
+                s4.x = fmaf(v4[u].x, w4, s4.x); s4.y = fmaf(v4[u].y, w4, s4.y);
+                s4.z = fmaf(v4[u].z, w4, s4.z); s4.w = fmaf(v4[u].w, w4, s4.w);
+              }
+            }
+            for (int j = part + MAXB * SPLIT; j < nparts; j += SPLIT) {
+              const float4 x4 = __ldcg(reinterpret_cast<const float4*>(
+                  pacc + (long long)(pbase + j) * G * D) + ch);
+              const float w4 = ssc[j * G + hch];
+              s4.x = fmaf(x4.x, w4, s4.x); s4.y = fmaf(x4.y, w4, s4.y);
+              s4.z = fmaf(x4.z, w4, s4.z); s4.w = fmaf(x4.w, w4, s4.w);
+            }
+            if (part > 0) scomb[(part - 1) * NCH + ch] = s4;
+          }
+          __syncthreads();
+          if (part == 0) {
+            for (int p2 = 1; p2 < SPLIT; ++p2) {
+              const float4 o4 = scomb[(p2 - 1) * NCH + ch];
+              s4.x += o4.x; s4.y += o4.y; s4.z += o4.z; s4.w += o4.w;
+            }
+            const int dd = (ch * 4) % D;
+            const float mt = stot[hch], lt = stot[G + hch];
+            const float inv = lt > 0.f ? 1.f / lt : 0.f;
+            const long long orow = ((long long)b * hq + hglob0 + hch) * D + dd;
+            outp[orow + 0] = (T)(s4.x * inv);
+            outp[orow + 1] = (T)(s4.y * inv);
+            outp[orow + 2] = (T)(s4.z * inv);
+            outp[orow + 3] = (T)(s4.w * inv);
+            if (dd == 0 && a.lse)
+              a.lse[(long long)b * hq + hglob0 + hch] =
+                  lt > 0.f ? (mt + fast_log2(lt)) * 0.69314718055994531f : -INFINITY;
+          }
         }
-        if (tid == 0) a.tickets[sigma] = 0;
+        if (tid == 0) {
+          a.tickets[sigma] = 0;
+          if (aligned) a.dyn[sigma] = 0;
+        }
       }
+    } else if (aligned && tid == 0) {
+      a.dyn[sigma] = 0;     // this CTA alone worked the segment
     }
     __syncthreads();
 
@@ -602,8 +905,12 @@ attn_kernel(const AttnArgs a) {
 
 template <typename T, int D, int G>
 struct Shape {
-  static constexpr int W = (sizeof(T) * D >= 512) ? 4 : 6;   // warps per CTA
-  static constexpr int NS = 2;                                // stages per warp
+  // warps per CTA: 16 KB tiles (fp32, d = 128) get fewer warps to fit stages
+  static constexpr int W = (sizeof(T) * D >= 512) ? 4 : ODA_ATTN_WARPS;
+  static constexpr int NS = ODA_ATTN_STAGES;                  // stages per warp
+  // smallest share of tiles a CTA takes, so a short launch uses fewer CTAs
+  static constexpr int MIN_TILES_RING = W * ODA_RING_TILES_PER_WARP;
+  static constexpr int MIN_TILES_FULL = W * ODA_FULL_TILES_PER_WARP;
 };
 
 template <typename T, int D, int G, bool RING>
@@ -611,11 +918,12 @@ size_t smem_bytes(int max_batch) {
   constexpr int W = Shape<T, D, G>::W, NS = Shape<T, D, G>::NS;
   constexpr size_t TILE_BYTES = 2 * ODA_TILE * D * sizeof(T);
   size_t s = (size_t)W * NS * TILE_BYTES;
+  s += (size_t)W * G * (D + 2) * 4 + 4;
   s += (size_t)W * NS * 8;
-  s += (size_t)W * 16 * G * 4;
-  s += (size_t)W * G * (D + 2) * 4;
-  s += (size_t)(3 * max_batch + 1) * 4;
-  s += 16;
+  s += (size_t)W * 32 * G * 4;
+  s += (size_t)(4 * max_batch + 2) * 4;
+  s += 16 + 64;
+  s += (size_t)W * NS * 4;
   s += (size_t)W * NS;
   return (s + 127) & ~(size_t)127;
 }
@@ -641,8 +949,9 @@ template <typename T, int D, int G, bool RING>
 oda_status launch_one(oda_ctx* ctx, const AttnArgs& a, int ctas, cudaStream_t st) {
   auto k = kernel_ptr<T, D, G, RING>();
   const size_t sm = smem_bytes<T, D, G, RING>(ctx->cfg.max_batch);
-  k<<<ctas, Shape<T, D, G>::W * 32, sm, st>>>(a);
-  return cudaGetLastError() == cudaSuccess ? ODA_OK : ODA_ERR_CUDA;
+  return launch_pdl(k, dim3(ctas), dim3(Shape<T, D, G>::W * 32), sm, st, a) == cudaSuccess
+             ? ODA_OK
+             : ODA_ERR_CUDA;
 }
 
 template <bool RING, typename F>
@@ -650,6 +959,11 @@ oda_status dispatch(const oda_config& c, F&& f) {
   const int G = c.hq / c.hkv;
 #define ODA_CASE(TT, DD, GG)                                                     \
   if (c.head_dim == DD && G == GG) return f.template operator()<TT, DD, GG, RING>();
+#ifdef ODA_ATTN_HOT_ONLY  // measurement builds: only the bf16, d = 128, G = 2 kernels
+  if (c.dtype == ODA_BF16) {
+    ODA_CASE(__nv_bfloat16, 128, 2)
+  }
+#else
   if (c.dtype == ODA_BF16) {
     ODA_CASE(__nv_bfloat16, 128, 2) ODA_CASE(__nv_bfloat16, 128, 1) ODA_CASE(__nv_bfloat16, 128, 4)
     ODA_CASE(__nv_bfloat16, 64, 2) ODA_CASE(__nv_bfloat16, 64, 1) ODA_CASE(__nv_bfloat16, 64, 4)
@@ -657,6 +971,7 @@ oda_status dispatch(const oda_config& c, F&& f) {
     ODA_CASE(float, 128, 2) ODA_CASE(float, 128, 1) ODA_CASE(float, 128, 4)
     ODA_CASE(float, 64, 2) ODA_CASE(float, 64, 1) ODA_CASE(float, 64, 4)
   }
+#endif
 #undef ODA_CASE
   return ODA_ERR_SHAPE;
 }
@@ -678,7 +993,7 @@ struct Launch {
   template <typename T, int D, int G, bool RING>
   oda_status operator()() {
     AttnArgs b = *a;
-    b.min_tiles_per_cta = Shape<T, D, G>::W;
+    b.min_tiles_per_cta = RING ? Shape<T, D, G>::MIN_TILES_RING : Shape<T, D, G>::MIN_TILES_FULL;
     return launch_one<T, D, G, RING>(ctx, b, RING ? ctx->attn_ctas_local : ctx->attn_ctas_full,
                                      st);
   }
@@ -725,7 +1040,9 @@ oda_status launch_attn(oda_ctx* ctx, bool ring_mode, int layer, const void* q,
   a.max_batch = c.max_batch;
   a.qscale = 1.4426950408889634f / sqrtf((float)c.head_dim);
   a.partials = ctx->partials;
+  a.max_parts = ctx->max_parts;
   a.tickets = ctx->tickets;
+  a.dyn = ctx->tickets + (size_t)c.max_batch * c.hkv;
   a.err = ctx->err;
   if (ring_mode) return dispatch<true>(c, Launch{ctx, &a, st, true});
   return dispatch<false>(c, Launch{ctx, &a, st, false});
@@ -758,7 +1075,7 @@ constexpr int kStaticMaxCtas = 512;            // persistent grid cap
 constexpr int kStaticMaxDevices = 64;
 
 static __device__ __align__(256) float g_static_partials[kStaticPartialFloats];
-static __device__ __align__(256) int g_static_tickets[kStaticMaxSegments];
+static __device__ __align__(256) int g_static_tickets[2 * kStaticMaxSegments];
 static __device__ __align__(256) int g_static_err[1];
 
 struct StaticDevice {
@@ -813,10 +1130,12 @@ struct LaunchStatic {
     const long long need = (long long)(ctas + B * a->hkv) * G * (D + 2);
     if (need > kStaticPartialFloats) return ODA_ERR_SHAPE;
     AttnArgs b = *a;
-    b.min_tiles_per_cta = Shape<T, D, G>::W;
+    b.max_parts = kStaticPartialFloats / (G * (D + 2));
+    b.min_tiles_per_cta = Shape<T, D, G>::MIN_TILES_FULL;
     b.max_batch = max_batch;
-    k<<<ctas, Shape<T, D, G>::W * 32, sm, st>>>(b);
-    return cudaGetLastError() == cudaSuccess ? ODA_OK : ODA_ERR_CUDA;
+    return launch_pdl(k, dim3(ctas), dim3(Shape<T, D, G>::W * 32), sm, st, b) == cudaSuccess
+               ? ODA_OK
+               : ODA_ERR_CUDA;
   }
 };
 
@@ -843,8 +1162,10 @@ extern "C" oda_status oda_full_attn_gated_static(const oda_config* cfg, int laye
   oda_status s = static_setup(dev, &sd);
   if (s != ODA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  // tickets must start at zero; a call that gave up early may have left some set
-  if (cudaMemsetAsync(sd->tickets, 0, sizeof(int) * (size_t)B * cfg->hkv, st) != cudaSuccess)
+  // tickets and the dynamic tile counters must start at zero; a call that
+  // gave up early may have left some set
+  if (cudaMemsetAsync(sd->tickets, 0, sizeof(int) * 2 * (size_t)kStaticMaxSegments, st) !=
+      cudaSuccess)
     return ODA_ERR_CUDA;
   AttnArgs a;
   a.q = q;
@@ -867,6 +1188,7 @@ extern "C" oda_status oda_full_attn_gated_static(const oda_config* cfg, int laye
   a.qscale = 1.4426950408889634f / sqrtf((float)cfg->head_dim);
   a.partials = sd->partials;
   a.tickets = sd->tickets;
+  a.dyn = sd->tickets + kStaticMaxSegments;
   a.err = err ? err : sd->err;
   return dispatch<false>(*cfg, LaunchStatic{&a, sd->num_sms, cfg->max_batch, B, st});
 }

@@ -22,6 +22,8 @@ gate_kernel(const float* __restrict__ scores, float theta, int B, uint8_t* __res
             cudaGraphConditionalHandle cond, int set_cond) {
   __shared__ int warp_counts[32];
   __shared__ int warp_base[33];
+  pdl_wait();
+  pdl_launch_dependents();
   const int tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
   bool f = false;
@@ -61,9 +63,11 @@ oda_status launch_gate(oda_ctx* ctx, const float* scores, float theta, int B, ui
                        unsigned long long cond_handle, bool set_cond) {
   (void)ctx;
   const int threads = ((B + 31) / 32) * 32 > 0 ? ((B + 31) / 32) * 32 : 32;
-  gate_kernel<<<1, threads, 0, st>>>(scores, theta, B, flags, idx, count,
-                                     (cudaGraphConditionalHandle)cond_handle, set_cond ? 1 : 0);
-  return cudaGetLastError() == cudaSuccess ? ODA_OK : ODA_ERR_CUDA;
+  return launch_pdl(gate_kernel, dim3(1), dim3(threads), 0, st, scores, theta, B, flags, idx,
+                    count, (cudaGraphConditionalHandle)cond_handle, set_cond ? 1 : 0) ==
+                 cudaSuccess
+             ? ODA_OK
+             : ODA_ERR_CUDA;
 }
 
 }  // namespace oda_impl

@@ -35,6 +35,8 @@ __device__ __forceinline__ long long ring_slot_off(int slot, int kv, int row_byt
 }
 
 __global__ void append_kernel(const AppendArgs a) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int chunks = a.row_bytes / 16;
   const long long total = (long long)a.nl * a.B * a.hkv * 2 * chunks;
   for (long long it = blockIdx.x * (long long)blockDim.x + threadIdx.x; it < total;
@@ -93,6 +95,8 @@ struct RingInitArgs {
 
 // One thread per 16-byte chunk of every (layer, row, head, K/V, slot).
 __global__ void ring_init_kernel(const RingInitArgs a) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int chunks = a.row_bytes / 16;
   const int slots = a.sink + a.window;
   const long long total = (long long)a.nl * a.B * a.hkv * 2 * slots * chunks;
@@ -173,8 +177,10 @@ oda_status launch_append(oda_ctx* ctx, int lb, int le, const void* k_new, const 
   a.ring_blocks = (int)ctx->lay.ring_blocks;
   a.err = ctx->err;
   const long long work = (long long)a.nl * B * c.hkv * 2 * (a.row_bytes / 16);
-  append_kernel<<<grid_for(work, 256, ctx->num_sms), 256, 0, st>>>(a);
-  return cudaGetLastError() == cudaSuccess ? ODA_OK : ODA_ERR_CUDA;
+  return launch_pdl(append_kernel, dim3(grid_for(work, 256, ctx->num_sms)), dim3(256), 0, st, a) ==
+                 cudaSuccess
+             ? ODA_OK
+             : ODA_ERR_CUDA;
 }
 
 oda_status launch_ring_init(oda_ctx* ctx, int lb, int le, const int32_t* seq_lens,
@@ -201,8 +207,10 @@ oda_status launch_ring_init(oda_ctx* ctx, int lb, int le, const int32_t* seq_len
   a.err = ctx->err;
   const long long work =
       (long long)a.nl * B * c.hkv * 2 * (c.sink + c.window) * (a.row_bytes / 16);
-  ring_init_kernel<<<grid_for(work, 256, ctx->num_sms), 256, 0, st>>>(a);
-  return cudaGetLastError() == cudaSuccess ? ODA_OK : ODA_ERR_CUDA;
+  return launch_pdl(ring_init_kernel, dim3(grid_for(work, 256, ctx->num_sms)), dim3(256), 0, st,
+                    a) == cudaSuccess
+             ? ODA_OK
+             : ODA_ERR_CUDA;
 }
 
 }  // namespace oda_impl

@@ -5,6 +5,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/oda.h"
 
 #define ODA_TILE 16  // tokens per paged block / ring tile
@@ -18,7 +20,8 @@ struct oda_ctx {
   int attn_ctas_full;        // persistent grid of the Full attention kernel
   int max_parts;             // capacity of the partials buffer (in partials)
   float* partials;           // [max_parts][G][d+2]
-  int* tickets;              // [max_batch * hkv], zero between launches
+  int* tickets;              // [2][max_batch * hkv]: merge tickets, dynamic tile counters;
+                             // zero between launches
   int* err;                  // device sticky error word
   int* recall_tickets;       // recall-head split reduction counters
   float* recall_partials;    // recall-head split partials
@@ -131,6 +134,34 @@ __device__ __forceinline__ float fast_log2(float x) {
 __device__ __forceinline__ void bf16x2_to_f32(uint32_t w, float& lo, float& hi) {
   lo = __uint_as_float(w << 16);
   hi = __uint_as_float(w & 0xFFFF0000u);
+}
+
+// Programmatic dependent launch: a kernel launched with
+// launch_pdl may be scheduled while its predecessor in the stream is still
+// running; pdl_wait() blocks until that predecessor has completed and its
+// writes are visible, so every kernel calls it before reading any input.
+// pdl_launch_dependents() lets the next kernel start being scheduled.
+__device__ __forceinline__ void pdl_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 }  // namespace oda

@@ -157,6 +157,8 @@ recall_kernel(const __grid_constant__ CUtensorMap tm_w1, const __grid_constant__
   uint32_t ncols = 32;
   while ((int)ncols < N) ncols <<= 1;
 
+  pdl_wait();
+  pdl_launch_dependents();
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(smem_addr(&full[s]), 1);
@@ -436,8 +438,10 @@ oda_status launch_recall(oda_ctx* ctx, const void* h_prev, const void* emb, cons
   a.stages = stages_for(N);
   const int U = a.MT * a.KB;
   const int grid = U < ctx->num_sms ? U : ctx->num_sms;
-  recall_kernel<<<grid, 192, smem_for(N, a.stages), st>>>(tw, t0, t1, t2, a);
-  return cudaGetLastError() == cudaSuccess ? ODA_OK : ODA_ERR_CUDA;
+  return launch_pdl(recall_kernel, dim3(grid), dim3(192), smem_for(N, a.stages), st, tw, t0, t1,
+                    t2, a) == cudaSuccess
+             ? ODA_OK
+             : ODA_ERR_CUDA;
 }
 
 }  // namespace oda_impl
