@@ -3,6 +3,7 @@
 #include <string.h>
 
 #include "oda_internal.cuh"
+#include "plan.cuh"
 
 using namespace oda;
 
@@ -104,6 +105,11 @@ oda_status oda_create(const oda_config* cfg, oda_ctx** out) {
         cudaMemset(ctx->err, 0, sizeof(int)) != cudaSuccess)
       s = ODA_ERR_CUDA;
   }
+  if (s == ODA_OK &&
+      cudaMalloc(&ctx->plan_local,
+                 PlanLayout::ints(cfg->max_batch, ctx->attn_ctas_local) * sizeof(int)) !=
+          cudaSuccess)
+    s = ODA_ERR_CUDA;
   if (s == ODA_OK) s = oda_impl::recall_setup(ctx);
   if (s == ODA_OK && cudaDeviceSynchronize() != cudaSuccess) s = ODA_ERR_CUDA;
   if (s != ODA_OK) {
@@ -122,6 +128,7 @@ oda_status oda_destroy(oda_ctx* ctx) {
   cudaFree(ctx->err);
   cudaFree(ctx->recall_partials);
   cudaFree(ctx->recall_tickets);
+  cudaFree(ctx->plan_local);
   free(ctx);
   return ODA_OK;
 }

@@ -26,6 +26,7 @@
 #include <mutex>
 
 #include "oda_internal.cuh"
+#include "plan.cuh"
 
 using namespace oda;
 
@@ -76,6 +77,7 @@ struct AttnArgs {
   int max_parts;
   int* tickets;                 // per segment: CTAs done (reset by the last)
   int* dyn;                     // per segment: tiles handed out dynamically (reset by the last)
+  const int* plan;              // precomputed partition, or null: compute it here
   int* err;
 };
 
@@ -205,129 +207,47 @@ attn_kernel(const AttnArgs a) {
   float* pml = a.partials + (size_t)a.max_parts * G * D;            // [max_parts][G][2]
 
   // ------------------------------------------------------- rows, partition
-  // Warp 0 reads the rows, builds the tile prefix and works out this CTA's
-  // share of the tiles (lane-parallel divisions, no block barrier); one
-  // barrier then publishes the result to the other warps through sinfo.
-  //
-  // Partition. "Aligned" when the segments fit the grid: each segment gets
-  // its own CTAs in proportion to its length (at least one, at most one per
-  // min_tiles tiles) and every CTA works inside one segment, so no CTA
-  // finishes one segment's merge before starting the next. Otherwise the
-  // tile space is split evenly and a CTA may span several segments.
+  // Either read the plan another kernel wrote once for every launch that
+  // shares it (one round trip of independent loads), or work it out here on
+  // warp 0; one barrier then publishes it through sinfo.
   if (warp == 0) {
-    int nr;
-    if (RING) {
-      nr = a.B;
+    if (a.plan) {
+      const int* pl = a.plan;
+      const int mb = a.max_batch;
+      const int hv = lane < 8 ? __ldcg(pl + PlanLayout::head() + lane) : 0;
+      const int dv = (lane >= 8 && lane < 13)
+                         ? __ldcg(pl + PlanLayout::cta(mb) + 8 * (int)blockIdx.x + (lane - 8))
+                         : 0;
+      for (int i = lane; i < a.B; i += 32) {
+        rowb[i] = __ldcg(pl + PlanLayout::rowb(mb) + i);
+        rowt[i] = __ldcg(pl + PlanLayout::rowt(mb) + i);
+      }
+      for (int i = lane; i <= a.B; i += 32) rowstart[i] = __ldcg(pl + PlanLayout::rowstart(mb) + i);
+      if (lane < 4) sinfo[lane] = hv;                 // nr, tot, P, al
+      if (lane >= 8 && lane < 13) sinfo[4 + lane - 8] = dv;   // lo, hi, pbase, nparts, part
+      if (lane == 0) sinfo[9] = (int)blockIdx.x;
     } else {
-      nr = *reinterpret_cast<const volatile int32_t*>(a.count);
-      if (nr < 0 || nr > a.B) {
-        if (lane == 0 && blockIdx.x == 0) record_error(a.err, ODA_ERR_BOUNDS);
-        nr = nr < 0 ? 0 : a.B;
+      PlanIn pin;
+      pin.B = a.B;
+      pin.count = RING ? nullptr : a.count;
+      pin.idx = a.idx;
+      pin.seq_lens = a.seq_lens;
+      pin.hkv = a.hkv;
+      pin.sink = a.sink;
+      pin.window = a.window;
+      pin.max_blocks = a.max_blocks;
+      pin.min_tiles = a.min_tiles_per_cta;
+      pin.grid = (int)gridDim.x;
+      pin.err = a.err;
+      pin.report = blockIdx.x == 0;
+      const PlanHead h = plan_rows(pin, rowb, rowt, rowstart, rowcs);
+      if (lane == 0) {
+        int o[5];
+        plan_cta((int)blockIdx.x, h, rowstart, rowcs, a.hkv, o);
+        sinfo[0] = h.nr; sinfo[1] = h.tot; sinfo[2] = h.P; sinfo[3] = h.al;
+        sinfo[4] = o[0]; sinfo[5] = o[1]; sinfo[6] = o[2]; sinfo[7] = o[3]; sinfo[8] = o[4];
+        sinfo[9] = (int)blockIdx.x;
       }
-    }
-    int carry = 0;
-    for (int base = 0; base < nr; base += 32) {
-      const int i = base + lane;
-      int nt = 0;
-      // with B <= 32 every lane loads one row's length alongside the index,
-      // so the two loads overlap instead of chaining (all lanes shuffle)
-      const int tl = (a.B <= 32 && lane < a.B) ? a.seq_lens[lane] : 0;
-      const int bl = i < nr ? (RING ? i : a.idx[i]) : 0;
-      const bool okl = bl >= 0 && bl < a.B;
-      const int ts = __shfl_sync(0xffffffffu, tl, okl ? (bl & 31) : 0);
-      if (i < nr) {
-        const int t = !okl ? 0 : (a.B <= 32 ? ts : a.seq_lens[bl]);
-        if (!okl || t < 1) {
-          if (blockIdx.x == 0) record_error(a.err, ODA_ERR_BOUNDS);
-        } else if (RING) {
-          nt = (a.sink + min(t, a.window) + ODA_TILE - 1) / ODA_TILE;
-        } else {
-          nt = (t + ODA_TILE - 1) / ODA_TILE;
-          if (nt > a.max_blocks) {
-            if (blockIdx.x == 0) record_error(a.err, ODA_ERR_BOUNDS);
-            nt = 0;
-          }
-        }
-        rowb[i] = okl ? bl : 0;
-        rowt[i] = t;
-      }
-      int v = nt * a.hkv;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        int y = __shfl_up_sync(0xffffffffu, v, o);
-        if (lane >= o) v += y;
-      }
-      if (i < nr) rowstart[i + 1] = carry + v;
-      carry += __shfl_sync(0xffffffffu, v, 31);
-    }
-    __syncwarp();                               // rowstart[] visible to every lane
-    const int tot = carry;
-    int P = (int)gridDim.x;
-    if (tot > 0) P = min(P, max(1, (tot + a.min_tiles_per_cta - 1) / a.min_tiles_per_cta));
-    // per-row CTA counts of the aligned partition, their prefix, the worst load
-    int carry2 = 0, worst = 0;
-    for (int base = 0; base < nr; base += 32) {
-      const int i = base + lane;
-      int n = 0;
-      if (i < nr) {
-        const int nt = (rowstart[i + 1] - (i == 0 ? 0 : rowstart[i])) / a.hkv;
-        if (nt > 0) {
-          n = ((unsigned)nt < (1u << 31) / (unsigned)P)
-                  ? (int)(((unsigned)nt * (unsigned)P) / (unsigned)tot)
-                  : (int)(((long long)nt * P) / tot);
-          n = max(min(n, nt / a.min_tiles_per_cta), 1);
-          worst = max(worst, (nt + n - 1) / n);
-        }
-      }
-      int v = n * a.hkv;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        int y = __shfl_up_sync(0xffffffffu, v, o);
-        if (lane >= o) v += y;
-      }
-      if (i < nr) rowcs[i + 1] = carry2 + v;
-      carry2 += __shfl_sync(0xffffffffu, v, 31);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) worst = max(worst, __shfl_xor_sync(0xffffffffu, worst, o));
-    __syncwarp();
-    if (lane == 0) {
-      rowstart[0] = 0;
-      rowcs[0] = 0;
-      const int cta0 = (int)blockIdx.x;
-      // aligned only if it fits the grid and no CTA gets more than 1.2x the
-      // even share of tiles
-      const int even = tot > 0 ? (tot + P - 1) / P : 0;
-      const bool al = tot > 0 && carry2 <= (int)gridDim.x && 5 * worst <= 6 * even;
-      int lo_ = 0, hi_ = 0, pb = 0, np = 0, pa = 0, vc = cta0;
-      if (tot > 0 && al && cta0 < carry2) {
-        vc = cta0;
-        int r0 = 0, r1 = nr - 1;                     // row with rowcs[r0] <= vc < rowcs[r0+1]
-        while (r0 < r1) {
-          const int mid = (r0 + r1 + 1) >> 1;
-          if (rowcs[mid] <= vc) r0 = mid; else r1 = mid - 1;
-        }
-        const int nt = (rowstart[r0 + 1] - rowstart[r0]) / a.hkv;
-        const int n = (rowcs[r0 + 1] - rowcs[r0]) / a.hkv;
-        const int g = (vc - rowcs[r0]) / n, part = vc - rowcs[r0] - g * n;
-        const int s0a = rowstart[r0] + g * nt;
-        if ((unsigned)nt < (1u << 31) / (unsigned)(n + 1)) {
-          lo_ = s0a + (int)(((unsigned)part * (unsigned)nt) / (unsigned)n);
-          hi_ = s0a + (int)(((unsigned)(part + 1) * (unsigned)nt) / (unsigned)n);
-        } else {
-          lo_ = s0a + (int)(((long long)part * nt) / n);
-          hi_ = s0a + (int)(((long long)(part + 1) * nt) / n);
-        }
-        pb = rowcs[r0] + g * n;
-        np = n;
-        pa = part;
-      } else if (tot > 0 && !al && cta0 < P) {
-        lo_ = (int)(((long long)cta0 * tot) / P);
-        hi_ = (int)(((long long)(cta0 + 1) * tot) / P);
-      }
-      sinfo[0] = nr; sinfo[1] = tot; sinfo[2] = P; sinfo[3] = al ? 1 : 0;
-      sinfo[4] = lo_; sinfo[5] = hi_; sinfo[6] = pb; sinfo[7] = np; sinfo[8] = pa;
-      sinfo[9] = vc;
     }
   }
   __syncthreads();
@@ -1017,7 +937,7 @@ oda_status attn_setup(oda_ctx* ctx) {
 oda_status launch_attn(oda_ctx* ctx, bool ring_mode, int layer, const void* q,
                        const int32_t* seq_lens, const void* kv, const int32_t* block_table,
                        const int32_t* idx, const int32_t* count, void* out, float* lse, int B,
-                       cudaStream_t st) {
+                       cudaStream_t st, const int* plan) {
   const oda_config& c = ctx->cfg;
   AttnArgs a;
   a.q = q;
@@ -1043,9 +963,26 @@ oda_status launch_attn(oda_ctx* ctx, bool ring_mode, int layer, const void* q,
   a.max_parts = ctx->max_parts;
   a.tickets = ctx->tickets;
   a.dyn = ctx->tickets + (size_t)c.max_batch * c.hkv;
+  a.plan = plan;
   a.err = ctx->err;
   if (ring_mode) return dispatch<true>(c, Launch{ctx, &a, st, true});
   return dispatch<false>(c, Launch{ctx, &a, st, false});
+}
+
+struct MinTiles {
+  int* out;
+  template <typename T, int D, int G, bool RING>
+  oda_status operator()() {
+    *out = RING ? Shape<T, D, G>::MIN_TILES_RING : Shape<T, D, G>::MIN_TILES_FULL;
+    return ODA_OK;
+  }
+};
+
+int attn_min_tiles(oda_ctx* ctx, bool ring_mode) {
+  int v = 1;
+  if (ring_mode) dispatch<true>(ctx->cfg, MinTiles{&v});
+  else dispatch<false>(ctx->cfg, MinTiles{&v});
+  return v;
 }
 
 }  // namespace oda_impl
@@ -1189,6 +1126,7 @@ extern "C" oda_status oda_full_attn_gated_static(const oda_config* cfg, int laye
   a.partials = sd->partials;
   a.tickets = sd->tickets;
   a.dyn = sd->tickets + kStaticMaxSegments;
+  a.plan = nullptr;
   a.err = err ? err : sd->err;
   return dispatch<false>(*cfg, LaunchStatic{&a, sd->num_sms, cfg->max_batch, B, st});
 }

@@ -6,6 +6,7 @@
 // layers. Here one launch commits a whole range of layers: each thread moves
 // 16 bytes, so a step at batch 1 with 28 layers is one small launch.
 #include "oda_internal.cuh"
+#include "plan.cuh"
 
 using namespace oda;
 
@@ -25,6 +26,10 @@ struct AppendArgs {
   int lb, nl, B, hkv, row_bytes;  // row_bytes = d * elem_bytes
   int sink, window, ring_blocks;
   int* err;
+  int nblk_append;              // blocks doing the copies; one more writes the plan
+  int* plan;                    // Local partition of this step's rows, or null
+  PlanIn pin;
+  int max_batch;
 };
 
 // Byte offset of slot `slot`, K (kv=0) or V (kv=1), inside the (row, head)
@@ -35,12 +40,19 @@ __device__ __forceinline__ long long ring_slot_off(int slot, int kv, int row_byt
 }
 
 __global__ void append_kernel(const AppendArgs a) {
+  extern __shared__ int plan_smem[];
   pdl_wait();
   pdl_launch_dependents();
+  if ((int)blockIdx.x == a.nblk_append) {
+    // The Local partition depends only on the rows' positions, so it is
+    // worked out once here for every Local launch of the step.
+    plan_write(a.pin, a.max_batch, a.plan, plan_smem);
+    return;
+  }
   const int chunks = a.row_bytes / 16;
   const long long total = (long long)a.nl * a.B * a.hkv * 2 * chunks;
   for (long long it = blockIdx.x * (long long)blockDim.x + threadIdx.x; it < total;
-       it += (long long)gridDim.x * blockDim.x) {
+       it += (long long)a.nblk_append * blockDim.x) {
     long long r = it;
     const int ch = (int)(r % chunks); r /= chunks;
     const int kv = (int)(r % 2); r /= 2;
@@ -154,7 +166,7 @@ namespace oda_impl {
 
 oda_status launch_append(oda_ctx* ctx, int lb, int le, const void* k_new, const void* v_new,
                          const int32_t* seq_lens, const int32_t* block_table, void* kv_cache,
-                         void* ring, int B, cudaStream_t st) {
+                         void* ring, int B, cudaStream_t st, int* local_plan) {
   const oda_config& c = ctx->cfg;
   AppendArgs a;
   a.k_new = static_cast<const unsigned char*>(k_new);
@@ -177,8 +189,27 @@ oda_status launch_append(oda_ctx* ctx, int lb, int le, const void* k_new, const 
   a.ring_blocks = (int)ctx->lay.ring_blocks;
   a.err = ctx->err;
   const long long work = (long long)a.nl * B * c.hkv * 2 * (a.row_bytes / 16);
-  return launch_pdl(append_kernel, dim3(grid_for(work, 256, ctx->num_sms)), dim3(256), 0, st, a) ==
-                 cudaSuccess
+  a.nblk_append = grid_for(work, 256, ctx->num_sms);
+  a.plan = local_plan;
+  a.max_batch = c.max_batch;
+  size_t smem = 0;
+  if (local_plan) {
+    a.pin.B = B;
+    a.pin.count = nullptr;
+    a.pin.idx = nullptr;
+    a.pin.seq_lens = seq_lens;
+    a.pin.hkv = c.hkv;
+    a.pin.sink = c.sink;
+    a.pin.window = c.window;
+    a.pin.max_blocks = c.max_blocks_per_seq;
+    a.pin.min_tiles = attn_min_tiles(ctx, true);
+    a.pin.grid = ctx->attn_ctas_local;
+    a.pin.err = ctx->err;
+    a.pin.report = true;
+    smem = (size_t)(4 * c.max_batch + 2) * sizeof(int);
+  }
+  const int grid = a.nblk_append + (local_plan ? 1 : 0);
+  return launch_pdl(append_kernel, dim3(grid), dim3(256), smem, st, a) == cudaSuccess
              ? ODA_OK
              : ODA_ERR_CUDA;
 }

@@ -26,6 +26,7 @@ struct oda_ctx {
   int* recall_tickets;       // recall-head split reduction counters
   float* recall_partials;    // recall-head split partials
   int recall_parts_cap;      // capacity of recall_partials in floats
+  int* plan_local;           // partition shared by a step's Local launches
 };
 
 namespace oda {
@@ -170,14 +171,15 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
 namespace oda_impl {
 oda_status launch_append(oda_ctx* ctx, int lb, int le, const void* k_new, const void* v_new,
                          const int32_t* seq_lens, const int32_t* block_table, void* kv_cache,
-                         void* ring, int B, cudaStream_t st);
+                         void* ring, int B, cudaStream_t st, int* local_plan = nullptr);
 oda_status launch_ring_init(oda_ctx* ctx, int lb, int le, const int32_t* seq_lens,
                             const int32_t* block_table, const void* kv_cache, void* ring, int B,
                             cudaStream_t st);
 oda_status launch_attn(oda_ctx* ctx, bool ring_mode, int layer, const void* q,
                        const int32_t* seq_lens, const void* kv, const int32_t* block_table,
                        const int32_t* idx, const int32_t* count, void* out, float* lse, int B,
-                       cudaStream_t st);
+                       cudaStream_t st, const int* plan = nullptr);
+int attn_min_tiles(oda_ctx* ctx, bool ring_mode);
 oda_status attn_setup(oda_ctx* ctx);
 oda_status launch_gate(oda_ctx* ctx, const float* scores, float theta, int B, uint8_t* flags,
                        int32_t* idx, int32_t* count, cudaStream_t st,

@@ -265,13 +265,15 @@ recall_kernel(const __grid_constant__ CUtensorMap tm_w1, const __grid_constant__
         const int c_first = (int)(((long long)(seg_lo + 1) * P - 1) / U);
         const int c_last = (int)(((long long)seg_hi * P - 1) / U);
         const int nparts = c_last - c_first + 1;
-        float* mypart = a.partials + (size_t)(c + mt) * N * BM;
+        // partials are [CTA + m-tile][row m][N]: a row's N sums are contiguous
+        float* mypart = a.partials + ((size_t)(c + mt) * BM + m) * N;
         // TMEM -> registers -> partials (always written; the merge reads them)
         for (int n0 = 0; n0 < N; n0 += 16) {
           float v[16];
           tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)n0, v);
 #pragma unroll
-          for (int e = 0; e < 16; ++e) mypart[(size_t)(n0 + e) * BM + m] = v[e];
+          for (int e = 0; e < 16; e += 4)
+            *reinterpret_cast<float4*>(mypart + n0 + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
         }
         fence_before_sync();
         if (lane == 0) mbar_arrive(smem_addr(acc_empty));
@@ -291,14 +293,48 @@ recall_kernel(const __grid_constant__ CUtensorMap tm_w1, const __grid_constant__
           __threadfence();
           const float bias = a.b1[mt * BM + m];
           const float wo = a.w2[mt * BM + m];
-          for (int n = 0; n < N; ++n) {
-            float acc = 0.f;
-            for (int c2 = c_first; c2 <= c_last; ++c2)
-              acc += __ldcg(a.partials + ((size_t)(c2 + mt) * N + n) * BM + m);
-            float contrib = wo * gelu_erf(acc + bias);
+          for (int n0 = 0; n0 < N; n0 += 16) {
+            // row m's 16 sums of every partial: all loads in flight together
+            float4 s4[4];
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) contrib += __shfl_xor_sync(0xffffffffu, contrib, o);
-            if (lane == 0) red[ew * MAX_N + n] = contrib;
+            for (int e = 0; e < 4; ++e) s4[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+            constexpr int PB = 4;
+            for (int c0 = c_first; c0 <= c_last; c0 += PB) {
+              float4 v4[PB][4];
+#pragma unroll
+              for (int u = 0; u < PB; ++u)
+                if (c0 + u <= c_last) {
+                  const float4* src = reinterpret_cast<const float4*>(
+                      a.partials + ((size_t)(c0 + u + mt) * BM + m) * N + n0);
+#pragma unroll
+                  for (int e = 0; e < 4; ++e) v4[u][e] = __ldcg(src + e);
+                }
+#pragma unroll
+              for (int u = 0; u < PB; ++u)
+                if (c0 + u <= c_last) {
+#pragma unroll
+                  for (int e = 0; e < 4; ++e) {
+                    s4[e].x += v4[u][e].x; s4[e].y += v4[u][e].y;
+                    s4[e].z += v4[u][e].z; s4[e].w += v4[u][e].w;
+                  }
+                }
+            }
+            float contrib[16];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              contrib[4 * e + 0] = wo * gelu_erf(s4[e].x + bias);
+              contrib[4 * e + 1] = wo * gelu_erf(s4[e].y + bias);
+              contrib[4 * e + 2] = wo * gelu_erf(s4[e].z + bias);
+              contrib[4 * e + 3] = wo * gelu_erf(s4[e].w + bias);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+              for (int e = 0; e < 16; ++e) contrib[e] += __shfl_xor_sync(0xffffffffu, contrib[e], o);
+            if (lane == 0) {
+#pragma unroll
+              for (int e = 0; e < 16; ++e) red[ew * MAX_N + n0 + e] = contrib[e];
+            }
           }
           epi_bar();
           for (int n = tid - 64; n < N; n += 128) {
@@ -317,10 +353,35 @@ recall_kernel(const __grid_constant__ CUtensorMap tm_w1, const __grid_constant__
           epi_bar();
           if (sflag[1]) {
             __threadfence();
-            for (int n = tid - 64; n < a.B; n += 128) {
+            // every (m-tile, row) dot product loaded at once, summed in a
+            // fixed order: thread j takes row j % Bc and m-tiles j / Bc + k*step
+            const int j = tid - 64;
+            const int Bc = a.B < 128 ? a.B : 128;
+            const int step = 128 / Bc;
+            float* red2 = red;                         // [128] partial sums
+            for (int n0 = 0; n0 < a.B; n0 += Bc) {     // same trip count on every thread
+              const int n = n0 + j % Bc;
               float s = 0.f;
-              for (int t2 = 0; t2 < a.MT; ++t2) s += __ldcg(a.spart + (size_t)t2 * N + n);
-              a.scores[n] = s + a.b2;
+              if (j / Bc < step && n < a.B) {
+                float v[8];
+                int t2 = j / Bc;
+                for (; t2 + 7 * step < a.MT; t2 += 8 * step) {
+#pragma unroll
+                  for (int u = 0; u < 8; ++u) v[u] = __ldcg(a.spart + (size_t)(t2 + u * step) * N + n);
+#pragma unroll
+                  for (int u = 0; u < 8; ++u) s += v[u];
+                }
+                for (; t2 < a.MT; t2 += step) s += __ldcg(a.spart + (size_t)t2 * N + n);
+              }
+              epi_bar();
+              if (j / Bc < step) red2[j] = s;
+              epi_bar();
+              if (j < Bc && n < a.B) {
+                float tsum = 0.f;
+                for (int k = 0; k < step; ++k) tsum += red2[k * Bc + j];
+                a.scores[n] = tsum + a.b2;
+              }
+              epi_bar();
             }
             if (tid == 64) a.tickets[MAX_MT] = 0;
           }

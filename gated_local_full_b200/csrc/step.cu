@@ -40,14 +40,15 @@ oda_status pre_part(oda_ctx* ctx, const oda_step_desc* d, cudaStream_t st,
   const oda_config& c = ctx->cfg;
   const size_t eb = (size_t)ctx->lay.elem_bytes;
   oda_status s = oda_impl::launch_append(ctx, 0, c.layers, d->k_new, d->v_new, d->seq_lens,
-                                         d->block_table, d->kv_cache, d->ring, d->B, st);
+                                         d->block_table, d->kv_cache, d->ring, d->B, st,
+                                         ctx->plan_local);
   if (s != ODA_OK) return s;
   for (int l = 0; l < c.layers; ++l) {
     const size_t qo = (size_t)l * layer_elems(ctx, d->B, c.hq) * eb;
     float* lse = d->lse ? d->lse + (size_t)l * d->B * c.hq : nullptr;
     s = oda_impl::launch_attn(ctx, true, l, static_cast<const char*>(d->q) + qo, d->seq_lens,
                               d->ring, nullptr, nullptr, nullptr,
-                              static_cast<char*>(d->out) + qo, lse, d->B, st);
+                              static_cast<char*>(d->out) + qo, lse, d->B, st, ctx->plan_local);
     if (s != ODA_OK) return s;
   }
   if (d->W1) {
