@@ -25,6 +25,9 @@
 //     segment's ticket merges them and writes the output.
 #include <mutex>
 
+#include <cooperative_groups.h>
+#include <stdlib.h>
+
 #include "oda_internal.cuh"
 #include "plan.cuh"
 
@@ -78,6 +81,7 @@ struct AttnArgs {
   int* tickets;                 // per segment: CTAs done (reset by the last)
   int* dyn;                     // per segment: tiles handed out dynamically (reset by the last)
   const int* plan;              // precomputed partition, or null: compute it here
+  int cluster;                  // cluster mode: CTAs per segment (= cluster size)
   int* err;
 };
 
@@ -168,7 +172,7 @@ struct Geom {
   static_assert(LPR == 8 || LPR == 16 || LPR == 32, "row must be 128, 256 or 512 bytes");
 };
 
-template <typename T, int D, int G, int W, int NS, bool RING>
+template <typename T, int D, int G, int W, int NS, bool RING, bool CL>
 __global__ void __launch_bounds__(W * 32, 2)
 attn_kernel(const AttnArgs a) {
   using Gm = Geom<T, D, G>;
@@ -192,6 +196,8 @@ attn_kernel(const AttnArgs a) {
   int* sinfo = sflag + 4;                                          // [16] partition of this CTA
   int* stile = sinfo + 16;                                         // [W][NS] tile of each stage
   unsigned char* badst = reinterpret_cast<unsigned char*>(stile + W * NS);  // [W][NS]
+  float* cst = reinterpret_cast<float*>(
+      (reinterpret_cast<uintptr_t>(badst + W * NS) + 15) & ~uintptr_t(15));  // CL: [G][D+2]
 
   const int tid = threadIdx.x;
   const int lane = tid & 31;
@@ -211,7 +217,30 @@ attn_kernel(const AttnArgs a) {
   // shares it (one round trip of independent loads), or work it out here on
   // warp 0; one barrier then publishes it through sinfo.
   if (warp == 0) {
-    if (a.plan) {
+    if (CL) {
+      // cluster mode: segment = cluster, tiles split evenly over its ranks
+      if (lane == 0) {
+        const int cs = a.cluster;
+        const int sg = (int)blockIdx.x / cs, rank = (int)blockIdx.x % cs;
+        const int b = sg / a.hkv, g = sg % a.hkv;
+        const bool okb = b < a.B;
+        const int t = okb ? a.seq_lens[b] : 0;
+        int nt = 0;
+        if (t < 1 || !okb) {
+          if (blockIdx.x == 0) record_error(a.err, ODA_ERR_BOUNDS);
+        } else {
+          nt = (a.sink + min(t, a.window) + ODA_TILE - 1) / ODA_TILE;
+        }
+        rowb[0] = okb ? b : 0;
+        rowt[0] = t;
+        rowstart[0] = 0;
+        rowstart[1] = nt * a.hkv;
+        sinfo[0] = 1; sinfo[1] = nt * a.hkv; sinfo[2] = (int)gridDim.x; sinfo[3] = 1;
+        sinfo[4] = g * nt + (rank * nt) / cs;
+        sinfo[5] = g * nt + ((rank + 1) * nt) / cs;
+        sinfo[6] = 0; sinfo[7] = cs; sinfo[8] = rank; sinfo[9] = (int)blockIdx.x;
+      }
+    } else if (a.plan) {
       const int* pl = a.plan;
       const int mb = a.max_batch;
       const int hv = lane < 8 ? __ldcg(pl + PlanLayout::head() + lane) : 0;
@@ -258,7 +287,13 @@ attn_kernel(const AttnArgs a) {
   int lo = sinfo[4], hi = sinfo[5];
   const int pbase_al = sinfo[6], nparts_al = sinfo[7], part_al = sinfo[8], vcta = sinfo[9];
   const int cta = (int)blockIdx.x;
-  if (nrows == 0 || total == 0 || lo >= hi) return;
+  // (cluster mode never leaves early: every CTA takes part in the merge)
+  const bool has_work = nrows > 0 && total > 0 && lo < hi;
+  if (!CL && !has_work) return;
+  if (CL && !has_work) {
+    for (int i = tid; i < G * (D + 2); i += W * 32)
+      cst[i] = (i % (D + 2)) == D ? -INFINITY : 0.f;   // empty state: m = -inf, l = acc = 0
+  } else {
 
   // K/V is read once per launch: stream it through L2 (the ring too, so no
   // layer's window stays resident from one step to the next)
@@ -279,7 +314,7 @@ attn_kernel(const AttnArgs a) {
   const int seg_s0 = prod.s1 - prod.nt;
   const int sigma0 = prod.i * a.hkv + prod.g;
   int pool0 = seg_nt;                        // first pool tile (relative); == nt: no pool
-  if (aligned && seg_nt >= 8 * nparts_al * W) {
+  if (!CL && aligned && seg_nt >= 8 * nparts_al * W) {
     pool0 = seg_nt - max(2 * nparts_al * W, seg_nt * ODA_POOL_PERCENT / 100);
     // static share of this CTA within [0, pool0)
     lo = seg_s0 + (int)(((long long)part_al * pool0) / nparts_al);
@@ -605,6 +640,29 @@ attn_kernel(const AttnArgs a) {
     }
     __syncthreads();
 
+    if constexpr (CL) {
+      // cluster mode: this CTA's merged state goes to shared memory, where
+      // cluster rank 0 reads it (one segment per CTA, so the loop ends here)
+      for (int o = tid; o < G * D; o += W * 32) {
+        const int h = o / D, dd = o % D;
+        float mt = -INFINITY;
+        for (int w2 = 0; w2 < W; ++w2) mt = fmaxf(mt, wstate[(w2 * G + h) * (D + 2) + D]);
+        float lt = 0.f, at = 0.f;
+        if (mt != -INFINITY) {
+          for (int w2 = 0; w2 < W; ++w2) {
+            const float* st = wstate + (w2 * G + h) * (D + 2);
+            if (st[D] == -INFINITY) continue;
+            const float sc2 = fast_exp2(st[D] - mt);
+            lt += st[D + 1] * sc2;
+            at += st[dd] * sc2;
+          }
+        }
+        cst[h * (D + 2) + dd] = at;
+        if (dd == 0) { cst[h * (D + 2) + D] = mt; cst[h * (D + 2) + D + 1] = lt; }
+      }
+      break;
+    }
+
     const int sigma = seg.i * a.hkv + seg.g;
     // the segment's partials are pbase .. pbase+nparts-1; this CTA writes mypart
     int pbase, nparts, mypart;
@@ -821,6 +879,62 @@ attn_kernel(const AttnArgs a) {
       }
     }
   }
+  }  // has_work
+
+  if constexpr (CL) {
+    // Cluster rank 0 merges the cluster's states through distributed shared
+    // memory: per query head, one warp finds the overall max and each rank's
+    // scale, then every output element sums the ranks' accumulators.
+    namespace cg = cooperative_groups;
+    cg::cluster_group cl = cg::this_cluster();
+    cl.sync();
+    if (cl.block_rank() == 0) {
+      constexpr int MAXC = 16;
+      const int cs = a.cluster;
+      const int sg = (int)blockIdx.x / cs;
+      const int b = rowb[0], g = sg % a.hkv;
+      float* sc = wstate;                        // [MAXC][G] scales
+      float* tt = wstate + MAXC * G;             // [2G] m_tot, l_tot
+      if (warp < G) {
+        const int h = warp;
+        float m = -INFINITY, l = 0.f;
+        if (lane < cs) {
+          const float* pr = cl.map_shared_rank(cst, lane);
+          m = pr[h * (D + 2) + D];
+          l = pr[h * (D + 2) + D + 1];
+        }
+        float mx = m;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        const float s2 = (m == -INFINITY || mx == -INFINITY) ? 0.f : fast_exp2(m - mx);
+        if (lane < cs) sc[lane * G + h] = s2;
+        float ls = l * s2;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
+        if (lane == 0) { tt[h] = mx; tt[G + h] = ls; }
+      }
+      __syncthreads();
+      T* outp = reinterpret_cast<T*>(a.out);
+      for (int o = tid; o < G * D; o += W * 32) {
+        const int h = o / D, dd = o % D;
+        float v[MAXC];
+#pragma unroll
+        for (int r = 0; r < MAXC; ++r)
+          v[r] = r < cs ? cl.map_shared_rank(cst, r)[h * (D + 2) + dd] : 0.f;
+        float at = 0.f;
+#pragma unroll
+        for (int r = 0; r < MAXC; ++r)
+          if (r < cs) at = fmaf(v[r], sc[r * G + h], at);
+        const float mt = tt[h], lt = tt[G + h];
+        const long long orow = ((long long)b * hq + g * G + h) * D;
+        outp[orow + dd] = (T)(lt > 0.f ? at / lt : 0.f);
+        if (dd == 0 && a.lse)
+          a.lse[(long long)b * hq + g * G + h] =
+              lt > 0.f ? (mt + fast_log2(lt)) * 0.69314718055994531f : -INFINITY;
+      }
+    }
+    cl.sync();                                   // ranks stay until rank 0 has read them
+  }
 }
 
 template <typename T, int D, int G>
@@ -845,12 +959,13 @@ size_t smem_bytes(int max_batch) {
   s += 16 + 64;
   s += (size_t)W * NS * 4;
   s += (size_t)W * NS;
+  s += 16 + (size_t)G * (D + 2) * 4;      // cluster mode: this CTA's merged state
   return (s + 127) & ~(size_t)127;
 }
 
-template <typename T, int D, int G, bool RING>
+template <typename T, int D, int G, bool RING, bool CL = false>
 auto kernel_ptr() {
-  return attn_kernel<T, D, G, Shape<T, D, G>::W, Shape<T, D, G>::NS, RING>;
+  return attn_kernel<T, D, G, Shape<T, D, G>::W, Shape<T, D, G>::NS, RING, CL>;
 }
 
 template <typename T, int D, int G, bool RING>
@@ -862,7 +977,62 @@ oda_status setup_one(oda_ctx* ctx, int& ctas) {
   ODA_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, Shape<T, D, G>::W * 32, sm));
   if (occ < 1) return ODA_ERR_SHAPE;
   ctas = ctx->num_sms * occ;
+  if (RING) {
+    // the cluster-merge variant of Local: largest cluster the GPU can hold
+    auto kc = kernel_ptr<T, D, G, true, true>();
+    ctx->local_cluster_max = 0;
+    if (cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(kc, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+      cudaGetLastError();
+      return ODA_OK;
+    }
+    // ODA_LOCAL_CLUSTER caps the cluster size (0 or 1: always the global merge)
+    int cap = 16;
+    if (const char* e = getenv("ODA_LOCAL_CLUSTER")) cap = atoi(e);
+    for (int cs = 16; cs >= 2; cs >>= 1) {
+      if (cs > cap) continue;
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(cs);
+      cfg.blockDim = dim3(Shape<T, D, G>::W * 32);
+      cfg.dynamicSmemBytes = sm;
+      cudaLaunchAttribute at[1];
+      at[0].id = cudaLaunchAttributeClusterDimension;
+      at[0].val.clusterDim.x = cs;
+      at[0].val.clusterDim.y = 1;
+      at[0].val.clusterDim.z = 1;
+      cfg.attrs = at;
+      cfg.numAttrs = 1;
+      int ncl = 0;
+      if (cudaOccupancyMaxActiveClusters(&ncl, kc, &cfg) == cudaSuccess && ncl > 0) {
+        ctx->local_cluster_max = cs;
+        break;
+      }
+      cudaGetLastError();
+    }
+  }
   return ODA_OK;
+}
+
+template <typename T, int D, int G>
+oda_status launch_cluster(oda_ctx* ctx, const AttnArgs& a, int grid, int cs, cudaStream_t st) {
+  auto k = kernel_ptr<T, D, G, true, true>();
+  const size_t sm = smem_bytes<T, D, G, true>(ctx->cfg.max_batch);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(Shape<T, D, G>::W * 32);
+  cfg.dynamicSmemBytes = sm;
+  cfg.stream = st;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = cs;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, k, a) == cudaSuccess ? ODA_OK : ODA_ERR_CUDA;
 }
 
 template <typename T, int D, int G, bool RING>
@@ -914,6 +1084,17 @@ struct Launch {
   oda_status operator()() {
     AttnArgs b = *a;
     b.min_tiles_per_cta = RING ? Shape<T, D, G>::MIN_TILES_RING : Shape<T, D, G>::MIN_TILES_FULL;
+    if (RING) {
+      // few segments: one cluster of cs CTAs per (row, KV head) segment,
+      // merged through distributed shared memory instead of global partials
+      const int S = b.B * b.hkv;
+      int cs = ctx->local_cluster_max;
+      while (cs >= 2 && S * cs > ctx->attn_ctas_local) cs >>= 1;
+      if (cs >= 2) {
+        b.cluster = cs;
+        return launch_cluster<T, D, G>(ctx, b, S * cs, cs, st);
+      }
+    }
     return launch_one<T, D, G, RING>(ctx, b, RING ? ctx->attn_ctas_local : ctx->attn_ctas_full,
                                      st);
   }
@@ -964,6 +1145,7 @@ oda_status launch_attn(oda_ctx* ctx, bool ring_mode, int layer, const void* q,
   a.tickets = ctx->tickets;
   a.dyn = ctx->tickets + (size_t)c.max_batch * c.hkv;
   a.plan = plan;
+  a.cluster = 0;
   a.err = ctx->err;
   if (ring_mode) return dispatch<true>(c, Launch{ctx, &a, st, true});
   return dispatch<false>(c, Launch{ctx, &a, st, false});
@@ -1127,6 +1309,7 @@ extern "C" oda_status oda_full_attn_gated_static(const oda_config* cfg, int laye
   a.tickets = sd->tickets;
   a.dyn = sd->tickets + kStaticMaxSegments;
   a.plan = nullptr;
+  a.cluster = 0;
   a.err = err ? err : sd->err;
   return dispatch<false>(*cfg, LaunchStatic{&a, sd->num_sms, cfg->max_batch, B, st});
 }

@@ -27,6 +27,7 @@ struct oda_ctx {
   float* recall_partials;    // recall-head split partials
   int recall_parts_cap;      // capacity of recall_partials in floats
   int* plan_local;           // partition shared by a step's Local launches
+  int local_cluster_max;     // largest cluster for the cluster-merge Local kernel (0: none)
 };
 
 namespace oda {

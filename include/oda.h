@@ -151,6 +151,11 @@ oda_status oda_ring_init(oda_ctx* ctx, int layer_begin, int layer_end,
  *   q     device [B][hq][d];  ring: all layers (layer 0 base)
  *   out   device [B][hq][d];  lse: device float [B][hq] or NULL
  *         (lse = log sum_j exp(q.k_j / sqrt d), natural log)
+ * When B*hkv segments times a cluster size fit one wave of CTAs, each
+ * (row, KV head) segment is split over one thread-block cluster and merged in
+ * distributed shared memory; otherwise the split is merged through the
+ * context's partials. The environment variable ODA_LOCAL_CLUSTER, read by
+ * oda_create, caps the cluster size (0: always the partials merge).
  */
 oda_status oda_local_attn(oda_ctx* ctx, int layer, const void* q,
                           const int32_t* seq_lens, const void* ring,

@@ -149,6 +149,24 @@ def test_edge_cases(torch, spec):
     assert ctx.get_device_error() == 0
 
 
+@pytest.mark.parametrize("cap", ["0", "2", "16"])
+def test_local_cluster_merge_and_global_merge(torch, monkeypatch, cap):
+    """Local through each merge of the split KV: the global partials merge
+    (cluster size cap 0) and the distributed-shared-memory cluster merge
+    (2 and 16 CTAs per segment). Rows span t <= s, t < s + w and t > s + w,
+    with ragged last tiles and ranks that get no tile at all."""
+    monkeypatch.setenv("ODA_LOCAL_CLUSTER", cap)
+    w = synth.custom("cluster", dtype="bf16", hq=8, hkv=4, window=200,
+                     t0=(3, 90, 205, 700), steps=2, fixed_scores=(0.0, 0.0, 0.0, 0.0))
+    ctx, dw = hx.setup(w)
+    b = _bufs(torch, w)
+    for step in range(w.steps):
+        local, lse_local = _run_step(ctx, dw, b, step)
+        torch.cuda.synchronize()
+        assert ctx.get_device_error() == 0
+        _check_step(torch, w, dw, b, step, local, lse_local)
+
+
 def test_all_rows_flagged_and_none(torch):
     w = synth.custom("flags", t0=(300, 200, 100), steps=1)
     ctx, dw = hx.setup(w)
