@@ -198,6 +198,8 @@ attn_kernel(const AttnArgs a) {
   unsigned char* badst = reinterpret_cast<unsigned char*>(stile + W * NS);  // [W][NS]
   float* cst = reinterpret_cast<float*>(
       (reinterpret_cast<uintptr_t>(badst + W * NS) + 15) & ~uintptr_t(15));  // CL: [G][D+2]
+  float* racc = cst + G * (D + 2);             // CL: [cs][G*D/cs] pushed accumulators
+  float* rml = racc + G * D;                   // CL: [16][G] pushed (m, l) pairs
 
   const int tid = threadIdx.x;
   const int lane = tid & 31;
@@ -207,6 +209,19 @@ attn_kernel(const AttnArgs a) {
   const int hq = a.hkv * G;
   if (tid < W * NS) mbar_init(smem_addr(&bars[tid]), 1);
   fence_mbar_init();
+  if constexpr (CL) {
+    cluster_arrive_relaxed();                    // "started": waited for before any remote store
+    // Before the dependency wait, warm L2 with this rank's share of a full
+    // ring (its share once t >= w). This reads no value: L2 is the point of
+    // coherence, so the loads after the wait still see every earlier write,
+    // and the prefetch overlaps the tail of the preceding kernel.
+    const int cs = a.cluster;
+    const int sg = (int)blockIdx.x / cs, rank = (int)blockIdx.x % cs;
+    const int rb = a.ring_blocks;
+    const int k0 = (rank * rb) / cs, k1 = ((rank + 1) * rb) / cs;
+    const T* base = reinterpret_cast<const T*>(a.kv) + (long long)sg * rb * TILE_ELEMS;
+    for (int k = k0 + tid; k < k1; k += W * 32) bulk_prefetch_l2(base + (long long)k * TILE_ELEMS, TILE_BYTES);
+  }
   pdl_wait();
   pdl_launch_dependents();
   float* pacc = a.partials;                                         // [max_parts][G][D]
@@ -882,58 +897,56 @@ attn_kernel(const AttnArgs a) {
   }  // has_work
 
   if constexpr (CL) {
-    // Cluster rank 0 merges the cluster's states through distributed shared
-    // memory: per query head, one warp finds the overall max and each rank's
-    // scale, then every output element sums the ranks' accumulators.
+    // Merge of the cluster's split KV. Each rank owns G*D/cs output elements;
+    // every rank pushes its accumulators for them, and its (m, l) per head,
+    // into the owner's shared memory (remote stores only), one cluster
+    // barrier publishes the stores, and each owner combines its elements
+    // from its own shared memory. No rank reads another rank's memory after
+    // that barrier, so ranks may exit as soon as they are done.
     namespace cg = cooperative_groups;
     cg::cluster_group cl = cg::this_cluster();
-    cl.sync();
-    if (cl.block_rank() == 0) {
-      constexpr int MAXC = 16;
-      const int cs = a.cluster;
-      const int sg = (int)blockIdx.x / cs;
-      const int b = rowb[0], g = sg % a.hkv;
-      float* sc = wstate;                        // [MAXC][G] scales
-      float* tt = wstate + MAXC * G;             // [2G] m_tot, l_tot
-      if (warp < G) {
-        const int h = warp;
-        float m = -INFINITY, l = 0.f;
-        if (lane < cs) {
-          const float* pr = cl.map_shared_rank(cst, lane);
-          m = pr[h * (D + 2) + D];
-          l = pr[h * (D + 2) + D + 1];
-        }
-        float mx = m;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        const float s2 = (m == -INFINITY || mx == -INFINITY) ? 0.f : fast_exp2(m - mx);
-        if (lane < cs) sc[lane * G + h] = s2;
-        float ls = l * s2;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
-        if (lane == 0) { tt[h] = mx; tt[G + h] = ls; }
-      }
-      __syncthreads();
-      T* outp = reinterpret_cast<T*>(a.out);
-      for (int o = tid; o < G * D; o += W * 32) {
-        const int h = o / D, dd = o % D;
-        float v[MAXC];
-#pragma unroll
-        for (int r = 0; r < MAXC; ++r)
-          v[r] = r < cs ? cl.map_shared_rank(cst, r)[h * (D + 2) + dd] : 0.f;
-        float at = 0.f;
-#pragma unroll
-        for (int r = 0; r < MAXC; ++r)
-          if (r < cs) at = fmaf(v[r], sc[r * G + h], at);
-        const float mt = tt[h], lt = tt[G + h];
-        const long long orow = ((long long)b * hq + g * G + h) * D;
-        outp[orow + dd] = (T)(lt > 0.f ? at / lt : 0.f);
-        if (dd == 0 && a.lse)
-          a.lse[(long long)b * hq + g * G + h] =
-              lt > 0.f ? (mt + fast_log2(lt)) * 0.69314718055994531f : -INFINITY;
-      }
+    constexpr int GD = G * D;
+    const int cs = a.cluster;
+    const int rank = (int)cl.block_rank();
+    const int per = GD / cs;
+    __syncthreads();                             // this CTA's state in cst is complete
+    cluster_wait();                              // every rank has started (arrived at entry)
+    for (int i = tid; i < GD; i += W * 32) {
+      const int h = i / D, dd = i % D;
+      float* dst = cl.map_shared_rank(racc, i / per);
+      dst[rank * per + i % per] = cst[h * (D + 2) + dd];
     }
-    cl.sync();                                   // ranks stay until rank 0 has read them
+    for (int j = tid; j < cs * G; j += W * 32) {
+      const int r2 = j / G, h = j % G;
+      float2* dst = reinterpret_cast<float2*>(cl.map_shared_rank(rml, r2));
+      dst[rank * G + h] = make_float2(cst[h * (D + 2) + D], cst[h * (D + 2) + D + 1]);
+    }
+    cluster_arrive();                            // release: the pushes above
+    cluster_wait();                              // acquire: every rank's pushes
+    const int b = rowb[0], g = ((int)blockIdx.x / cs) % a.hkv;
+    const float2* ml = reinterpret_cast<const float2*>(rml);
+    T* outp = reinterpret_cast<T*>(a.out);
+    for (int ol = tid; ol < per; ol += W * 32) {
+      const int o = rank * per + ol;
+      const int h = o / D, dd = o % D;
+      float mt = -INFINITY;
+      for (int r = 0; r < cs; ++r) mt = fmaxf(mt, ml[r * G + h].x);
+      float lt = 0.f, at = 0.f;
+      if (mt != -INFINITY) {
+        for (int r = 0; r < cs; ++r) {
+          const float2 v = ml[r * G + h];
+          if (v.x == -INFINITY) continue;
+          const float sc2 = fast_exp2(v.x - mt);
+          lt += v.y * sc2;
+          at += racc[r * per + ol] * sc2;
+        }
+      }
+      const long long orow = ((long long)b * hq + g * G + h) * D;
+      outp[orow + dd] = (T)(lt > 0.f ? at / lt : 0.f);
+      if (dd == 0 && a.lse)
+        a.lse[(long long)b * hq + g * G + h] =
+            lt > 0.f ? (mt + fast_log2(lt)) * 0.69314718055994531f : -INFINITY;
+    }
   }
 }
 
@@ -959,7 +972,7 @@ size_t smem_bytes(int max_batch) {
   s += 16 + 64;
   s += (size_t)W * NS * 4;
   s += (size_t)W * NS;
-  s += 16 + (size_t)G * (D + 2) * 4;      // cluster mode: this CTA's merged state
+  s += 16 + (size_t)(G * (D + 2) + G * D + 32 * G) * 4;   // cluster mode: state, merge buffers
   return (s + 127) & ~(size_t)127;
 }
 
