@@ -188,6 +188,37 @@ def peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
+KERNEL_SOURCES = ("attn.cu", "plan.cuh", "oda_internal.cuh")
+
+
+def kernel_src_sha1() -> str:
+    """Digest of the attention kernel's sources (what the ncu counters were taken on)."""
+    h = hashlib.sha1()
+    for f in KERNEL_SOURCES:
+        h.update(open(os.path.join(ROOT, "gated_local_full_b200", "csrc", f), "rb").read())
+    return h.hexdigest()
+
+
+def replay_seconds(torch, fn, stream) -> float:
+    """Device time of the launches `fn` makes: captured once in a CUDA graph,
+    replayed once to warm up, then timed between CUDA events on `stream`."""
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        fn()
+    stream.wait_stream(side)
+    with torch.cuda.stream(stream):
+        g.replay()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        g.replay()
+        b.record(stream)
+    torch.cuda.synchronize()
+    del g
+    return a.elapsed_time(b) / 1000.0
+
+
 def recorded_traffic():
     """Per-launch DRAM traffic of the Full-attention kernel from the committed
     ncu summary, if it was taken on the current kernel source."""
@@ -195,8 +226,7 @@ def recorded_traffic():
     if not os.path.exists(p):
         return None, None
     d = json.load(open(p))
-    src = open(os.path.join(ROOT, "gated_local_full_b200", "csrc", "attn.cu"), "rb").read()
-    if d.get("attn_cu_sha1") != hashlib.sha1(src).hexdigest():
+    if d.get("kernel_src_sha1") != kernel_src_sha1():
         return None, d
     return d.get("full_attn_traffic_bytes_per_launch_128k"), d
 
@@ -409,39 +439,36 @@ def run_oda(args, rank, ws, local):
     # flagged steps launch them; plain launches issue them every step
     launches = K * (w.layers + 4) + (n_flag if args.launch == "graph" else K) * w.layers
 
-    # ---- dominant kernel: Full attention, per-launch CUDA-event timing on this stream
+    # ---- dominant kernel: Full attention. As in a flagged step, the L layers'
+    # launches run back to back: the runs of up to 16 flagged steps are
+    # captured in one CUDA graph (no host launch cost between kernels), which
+    # is replayed between two CUDA events on this stream; the average launch
+    # duration is the replay's time over its launches.
     cnt1 = torch.ones(1, dtype=torch.int32, device="cuda")
     idx0 = torch.zeros(w.batch, dtype=torch.int32, device="cuda")
     outb = torch.empty_like(st.out[0])
     fl_steps = [i for i in timed if flags[i]][:16] or [timed[0]]
-    evs = []
-    for i in fl_steps:
-        q = st.record_view(recs, i, "q")
-        sl = st.record_view(recs, i, "seq_lens")
-        for l in range(w.layers):
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            ctx.full_attn_gated(l, q[l], sl, dw.block_table, dw.cache, idx0, cnt1, outb, None,
-                                w.batch)
-            b.record(stream)
-            evs.append((a, b, int(w.t0[0]) + i))
-    torch.cuda.synchronize()
-    durs = np.array([a.elapsed_time(b) / 1000.0 for a, b, _ in evs])
-    bytes_per = np.array([t * KV_BYTES_PER_TOKEN_LAYER for _, _, t in evs], dtype=np.float64)
-    full_gbs = float(bytes_per.mean() / durs.mean() / 1e9)
-    # Local attention launches, same method (information)
-    evl = []
-    for i in timed[:16]:
-        q = st.record_view(recs, i, "q")
-        sl = st.record_view(recs, i, "seq_lens")
-        for l in range(w.layers):
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            ctx.local_attn(l, q[l], sl, dw.ring, outb, None, w.batch)
-            b.record(stream)
-            evl.append((a, b))
-    torch.cuda.synchronize()
-    local_us = float(np.mean([a.elapsed_time(b) for a, b in evl]) * 1000.0)
+
+    def run_full():
+        for i in fl_steps:
+            q = st.record_view(recs, i, "q")
+            sl = st.record_view(recs, i, "seq_lens")
+            for l in range(w.layers):
+                ctx.full_attn_gated(l, q[l], sl, dw.block_table, dw.cache, idx0, cnt1, outb,
+                                    None, w.batch)
+
+    def run_local():
+        for i in timed[:16]:
+            q = st.record_view(recs, i, "q")
+            sl = st.record_view(recs, i, "seq_lens")
+            for l in range(w.layers):
+                ctx.local_attn(l, q[l], sl, dw.ring, outb, None, w.batch)
+
+    full_s, n_full = replay_seconds(torch, run_full, stream), len(fl_steps) * w.layers
+    local_s, n_local = replay_seconds(torch, run_local, stream), min(K, 16) * w.layers
+    full_bytes = sum((int(w.t0[0]) + i) * KV_BYTES_PER_TOKEN_LAYER for i in fl_steps) * w.layers
+    full_gbs = float(full_bytes / full_s / 1e9)
+    local_us = float(local_s / n_local * 1e6)
     hbm, hbm_kind = peaks()
     traffic, _ = recorded_traffic()
 
@@ -500,8 +527,10 @@ def run_oda(args, rank, ws, local):
                          "frac": full_gbs / hbm, "traffic": traffic,
                          "kernel": "attn_kernel<bf16,128,2,RING=false> (Full attention)",
                          "peak_kind": hbm_kind,
-                         "launches_timed": len(evs),
-                         "mean_launch_us": float(durs.mean() * 1e6)},
+                         "launches_timed": n_full,
+                         "timing": "CUDA events on the launching stream around a graph "
+                                   "replay of L back-to-back launches per flagged step",
+                         "mean_launch_us": float(full_s / n_full * 1e6)},
             "local_attn_mean_launch_us": local_us,
             "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks, "gpu_launches": launches,
             "device_error": err,

@@ -44,6 +44,9 @@ using namespace oda;
 #ifndef ODA_RING_TILES_PER_WARP
 #define ODA_RING_TILES_PER_WARP 1
 #endif
+#ifndef ODA_PREFETCH_TILES  // tiles per CTA warmed in L2 before the dependency wait
+#define ODA_PREFETCH_TILES 16
+#endif
 #ifndef ODA_POOL_PERCENT
 #define ODA_POOL_PERCENT 15
 #endif
@@ -115,6 +118,11 @@ __device__ __forceinline__ uint32_t range_bits(int lo, int hi, int base) {
   int h = min(max(hi - base, 0), 16);
   if (h <= l) return 0u;
   return ((1u << h) - 1u) & ~((1u << l) - 1u);
+}
+
+// Pool size of an aligned segment of nt tiles over np CTAs of W warps.
+__device__ __forceinline__ int pool_tiles(int nt, int np, int W) {
+  return max(2 * np * W, nt * ODA_POOL_PERCENT / 100);
 }
 
 // Segment cursor over the CTA's tile range [lo, hi): segment (i, g) covers
@@ -222,15 +230,102 @@ attn_kernel(const AttnArgs a) {
     const T* base = reinterpret_cast<const T*>(a.kv) + (long long)sg * rb * TILE_ELEMS;
     for (int k = k0 + tid; k < k1; k += W * 32) bulk_prefetch_l2(base + (long long)k * TILE_ELEMS, TILE_BYTES);
   }
+  // ------------------------------------------------------- rows, partition
+  // Either read the plan another kernel wrote once for every launch that
+  // shares it (one round trip of independent loads), or work it out here on
+  // warp 0; one barrier then publishes it through sinfo.
+  auto partition = [&](bool report) {          // warp 0, non-cluster modes
+    if (a.plan) {
+      const int* pl = a.plan;
+      const int mb = a.max_batch;
+      const int hv = lane < 8 ? __ldcg(pl + PlanLayout::head() + lane) : 0;
+      const int dv = (lane >= 8 && lane < 13)
+          ? __ldcg(pl + PlanLayout::cta(mb) + 8 * (int)blockIdx.x + (lane - 8))
+          : 0;
+      for (int i = lane; i < a.B; i += 32) {
+        rowb[i] = __ldcg(pl + PlanLayout::rowb(mb) + i);
+        rowt[i] = __ldcg(pl + PlanLayout::rowt(mb) + i);
+      }
+      for (int i = lane; i <= a.B; i += 32) rowstart[i] = __ldcg(pl + PlanLayout::rowstart(mb) + i);
+      if (lane < 4) sinfo[lane] = hv;                 // nr, tot, P, al
+      if (lane >= 8 && lane < 13) sinfo[4 + lane - 8] = dv;   // lo, hi, pbase, nparts, part
+      if (lane == 0) sinfo[9] = (int)blockIdx.x;
+    } else {
+      PlanIn pin;
+      pin.B = a.B;
+      pin.count = RING ? nullptr : a.count;
+      pin.idx = a.idx;
+      pin.seq_lens = a.seq_lens;
+      pin.hkv = a.hkv;
+      pin.sink = a.sink;
+      pin.window = a.window;
+      pin.max_blocks = a.max_blocks;
+      pin.min_tiles = a.min_tiles_per_cta;
+      pin.grid = (int)gridDim.x;
+      pin.err = a.err;
+      pin.report = report && blockIdx.x == 0;
+      const PlanHead h = plan_rows(pin, rowb, rowt, rowstart, rowcs);
+      if (lane == 0) {
+        int o[5];
+        plan_cta((int)blockIdx.x, h, rowstart, rowcs, a.hkv, o);
+        sinfo[0] = h.nr; sinfo[1] = h.tot; sinfo[2] = h.P; sinfo[3] = h.al;
+        sinfo[4] = o[0]; sinfo[5] = o[1]; sinfo[6] = o[2]; sinfo[7] = o[3]; sinfo[8] = o[4];
+        sinfo[9] = (int)blockIdx.x;
+      }
+    }
+  };
+
+#if ODA_PREFETCH_TILES > 0
+  static_assert(ODA_PREFETCH_TILES <= 32, "one prefetched tile per lane of warp 0");
+  if constexpr (!CL) {
+    // Before the dependency wait, warp 0 works out the partition from values
+    // that the preceding launch may still be writing, and warms L2 with the
+    // first tiles of this CTA's static share. Nothing read here is used after
+    // the wait (the partition is worked out again), and an L2 prefetch reads
+    // no value, so a stale guess only costs bandwidth; every address is
+    // bounds-checked like the loads proper.
+    if (warp == 0) {
+      partition(false);
+      __syncwarp();
+      const int nr = sinfo[0], tot = sinfo[1];
+      int plo = sinfo[4], phi = sinfo[5];
+      if (nr > 0 && nr <= a.B && tot > 0 && plo >= 0 && plo < phi && phi <= tot) {
+        Cursor c;
+        locate(rowstart, nr, a.hkv, plo, c);
+        const int nt = c.nt, s0 = c.s1 - c.nt, np = sinfo[7], pt = sinfo[8];
+        if (sinfo[3] && np > 0 && nt >= 8 * np * W) {
+          const int p0 = nt - pool_tiles(nt, np, W);
+          plo = s0 + (int)(((long long)pt * p0) / np);
+          phi = s0 + (int)(((long long)(pt + 1) * p0) / np);
+        }
+        const int k = plo + lane;
+        if (lane < ODA_PREFETCH_TILES && k < phi) {
+          Cursor ck;
+          locate(rowstart, nr, a.hkv, k, ck);
+          const int jt = k - (rowstart[ck.i] + ck.g * ck.nt);
+          const int b = rowb[ck.i];
+          const T* kb = reinterpret_cast<const T*>(a.kv);
+          const bool ok = b >= 0 && b < a.B && ck.g >= 0 && ck.g < a.hkv && jt >= 0;
+          if (RING) {
+            if (ok && jt < a.ring_blocks)
+              bulk_prefetch_l2(kb + (((long long)b * a.hkv + ck.g) * a.ring_blocks + jt) * TILE_ELEMS,
+                               TILE_BYTES);
+          } else if (ok && jt < a.max_blocks) {
+            const int blk = __ldcg(a.block_table + (long long)b * a.max_blocks + jt);
+            if (blk >= 0 && (long long)blk < a.num_blocks)
+              bulk_prefetch_l2(kb + ((long long)blk * a.hkv + ck.g) * TILE_ELEMS, TILE_BYTES);
+          }
+        }
+      }
+      __syncwarp();
+    }
+  }
+#endif
   pdl_wait();
   pdl_launch_dependents();
   float* pacc = a.partials;                                         // [max_parts][G][D]
   float* pml = a.partials + (size_t)a.max_parts * G * D;            // [max_parts][G][2]
 
-  // ------------------------------------------------------- rows, partition
-  // Either read the plan another kernel wrote once for every launch that
-  // shares it (one round trip of independent loads), or work it out here on
-  // warp 0; one barrier then publishes it through sinfo.
   if (warp == 0) {
     if (CL) {
       // cluster mode: segment = cluster, tiles split evenly over its ranks
@@ -255,43 +350,8 @@ attn_kernel(const AttnArgs a) {
         sinfo[5] = g * nt + ((rank + 1) * nt) / cs;
         sinfo[6] = 0; sinfo[7] = cs; sinfo[8] = rank; sinfo[9] = (int)blockIdx.x;
       }
-    } else if (a.plan) {
-      const int* pl = a.plan;
-      const int mb = a.max_batch;
-      const int hv = lane < 8 ? __ldcg(pl + PlanLayout::head() + lane) : 0;
-      const int dv = (lane >= 8 && lane < 13)
-                         ? __ldcg(pl + PlanLayout::cta(mb) + 8 * (int)blockIdx.x + (lane - 8))
-                         : 0;
-      for (int i = lane; i < a.B; i += 32) {
-        rowb[i] = __ldcg(pl + PlanLayout::rowb(mb) + i);
-        rowt[i] = __ldcg(pl + PlanLayout::rowt(mb) + i);
-      }
-      for (int i = lane; i <= a.B; i += 32) rowstart[i] = __ldcg(pl + PlanLayout::rowstart(mb) + i);
-      if (lane < 4) sinfo[lane] = hv;                 // nr, tot, P, al
-      if (lane >= 8 && lane < 13) sinfo[4 + lane - 8] = dv;   // lo, hi, pbase, nparts, part
-      if (lane == 0) sinfo[9] = (int)blockIdx.x;
     } else {
-      PlanIn pin;
-      pin.B = a.B;
-      pin.count = RING ? nullptr : a.count;
-      pin.idx = a.idx;
-      pin.seq_lens = a.seq_lens;
-      pin.hkv = a.hkv;
-      pin.sink = a.sink;
-      pin.window = a.window;
-      pin.max_blocks = a.max_blocks;
-      pin.min_tiles = a.min_tiles_per_cta;
-      pin.grid = (int)gridDim.x;
-      pin.err = a.err;
-      pin.report = blockIdx.x == 0;
-      const PlanHead h = plan_rows(pin, rowb, rowt, rowstart, rowcs);
-      if (lane == 0) {
-        int o[5];
-        plan_cta((int)blockIdx.x, h, rowstart, rowcs, a.hkv, o);
-        sinfo[0] = h.nr; sinfo[1] = h.tot; sinfo[2] = h.P; sinfo[3] = h.al;
-        sinfo[4] = o[0]; sinfo[5] = o[1]; sinfo[6] = o[2]; sinfo[7] = o[3]; sinfo[8] = o[4];
-        sinfo[9] = (int)blockIdx.x;
-      }
+      partition(true);
     }
   }
   __syncthreads();
@@ -330,7 +390,7 @@ attn_kernel(const AttnArgs a) {
   const int sigma0 = prod.i * a.hkv + prod.g;
   int pool0 = seg_nt;                        // first pool tile (relative); == nt: no pool
   if (!CL && aligned && seg_nt >= 8 * nparts_al * W) {
-    pool0 = seg_nt - max(2 * nparts_al * W, seg_nt * ODA_POOL_PERCENT / 100);
+    pool0 = seg_nt - pool_tiles(seg_nt, nparts_al, W);
     // static share of this CTA within [0, pool0)
     lo = seg_s0 + (int)(((long long)part_al * pool0) / nparts_al);
     hi = seg_s0 + (int)(((long long)(part_al + 1) * pool0) / nparts_al);

@@ -12,7 +12,9 @@
 // Aligned is used only if no CTA would get more than 1.2x the even share.
 //
 // plan_rows runs on warp 0 of a block and leaves the per-row arrays in shared
-// memory; plan_cta turns them into one CTA's share. The attention kernel can
+// memory; plan_cta turns them into one CTA's share. Its global loads bypass
+// L1 (ld.global.cg), so a guess made before a dependency wait leaves no stale
+// line behind for the loads after it. The attention kernel can
 // run both itself, or read a plan that another kernel wrote once for all the
 // launches that share it (the Local launches of a decode step).
 #pragma once
@@ -58,12 +60,12 @@ __device__ __forceinline__ PlanHead plan_rows(const PlanIn& p, int* rowb, int* r
     int nt = 0;
     // with B <= 32 every lane loads one row's length alongside the index,
     // so the two loads overlap instead of chaining (all lanes shuffle)
-    const int tl = (p.B <= 32 && lane < p.B) ? p.seq_lens[lane] : 0;
-    const int bl = i < nr ? (ring ? i : p.idx[i]) : 0;
+    const int tl = (p.B <= 32 && lane < p.B) ? __ldcg(p.seq_lens + lane) : 0;
+    const int bl = i < nr ? (ring ? i : __ldcg(p.idx + i)) : 0;
     const bool okl = bl >= 0 && bl < p.B;
     const int ts = __shfl_sync(0xffffffffu, tl, okl ? (bl & 31) : 0);
     if (i < nr) {
-      const int t = !okl ? 0 : (p.B <= 32 ? ts : p.seq_lens[bl]);
+      const int t = !okl ? 0 : (p.B <= 32 ? ts : __ldcg(p.seq_lens + bl));
       if (!okl || t < 1) {
         if (p.report) record_error(p.err, ODA_ERR_BOUNDS);
       } else if (ring) {
