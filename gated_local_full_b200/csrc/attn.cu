@@ -1020,9 +1020,19 @@ struct Shape {
   static constexpr int MIN_TILES_FULL = W * ODA_FULL_TILES_PER_WARP;
 };
 
-template <typename T, int D, int G, bool RING>
-size_t smem_bytes(int max_batch) {
-  constexpr int W = Shape<T, D, G>::W, NS = Shape<T, D, G>::NS;
+// Cluster-merge Local launches whose CTAs hold at most ODA_CL_WIDE_WARPS tiles
+// each (a full ring over a 16-CTA cluster) use one warp per tile and a single
+// stage, so no warp works two tiles in turn.
+#ifndef ODA_CL_WIDE_WARPS
+#define ODA_CL_WIDE_WARPS 9
+#endif
+struct ShapeWide {
+  static constexpr int W = ODA_CL_WIDE_WARPS;
+  static constexpr int NS = 1;
+};
+
+template <typename T, int D, int G, int W, int NS>
+size_t smem_bytes_wn(int max_batch) {
   constexpr size_t TILE_BYTES = 2 * ODA_TILE * D * sizeof(T);
   size_t s = (size_t)W * NS * TILE_BYTES;
   s += (size_t)W * G * (D + 2) * 4 + 4;
@@ -1036,9 +1046,56 @@ size_t smem_bytes(int max_batch) {
   return (s + 127) & ~(size_t)127;
 }
 
+template <typename T, int D, int G, bool RING>
+size_t smem_bytes(int max_batch) {
+  return smem_bytes_wn<T, D, G, Shape<T, D, G>::W, Shape<T, D, G>::NS>(max_batch);
+}
+
 template <typename T, int D, int G, bool RING, bool CL = false>
 auto kernel_ptr() {
   return attn_kernel<T, D, G, Shape<T, D, G>::W, Shape<T, D, G>::NS, RING, CL>;
+}
+
+// Cluster-merge Local kernel of shape (W, NS): sets its attributes and returns
+// the largest cluster size (16, 8, 4, 2) of which the GPU holds at least one
+// cluster, capped by ODA_LOCAL_CLUSTER; 0 if none. `ctas` receives the CTAs
+// one wave holds.
+template <typename T, int D, int G, int W, int NS>
+int cluster_setup(oda_ctx* ctx, int& ctas) {
+  auto kc = attn_kernel<T, D, G, W, NS, true, true>;
+  const size_t sm = smem_bytes_wn<T, D, G, W, NS>(ctx->cfg.max_batch);
+  ctas = 0;
+  int occ = 0;
+  if (cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) !=
+          cudaSuccess ||
+      cudaFuncSetAttribute(kc, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kc, W * 32, sm) != cudaSuccess ||
+      occ < 1) {
+    cudaGetLastError();
+    return 0;
+  }
+  ctas = ctx->num_sms * occ;
+  // ODA_LOCAL_CLUSTER caps the cluster size (0 or 1: always the global merge)
+  int cap = 16;
+  if (const char* e = getenv("ODA_LOCAL_CLUSTER")) cap = atoi(e);
+  for (int cs = 16; cs >= 2; cs >>= 1) {
+    if (cs > cap) continue;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(cs);
+    cfg.blockDim = dim3(W * 32);
+    cfg.dynamicSmemBytes = sm;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = cs;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    int ncl = 0;
+    if (cudaOccupancyMaxActiveClusters(&ncl, kc, &cfg) == cudaSuccess && ncl > 0) return cs;
+    cudaGetLastError();
+  }
+  return 0;
 }
 
 template <typename T, int D, int G, bool RING>
@@ -1051,49 +1108,22 @@ oda_status setup_one(oda_ctx* ctx, int& ctas) {
   if (occ < 1) return ODA_ERR_SHAPE;
   ctas = ctx->num_sms * occ;
   if (RING) {
-    // the cluster-merge variant of Local: largest cluster the GPU can hold
-    auto kc = kernel_ptr<T, D, G, true, true>();
-    ctx->local_cluster_max = 0;
-    if (cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) !=
-            cudaSuccess ||
-        cudaFuncSetAttribute(kc, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
-      cudaGetLastError();
-      return ODA_OK;
-    }
-    // ODA_LOCAL_CLUSTER caps the cluster size (0 or 1: always the global merge)
-    int cap = 16;
-    if (const char* e = getenv("ODA_LOCAL_CLUSTER")) cap = atoi(e);
-    for (int cs = 16; cs >= 2; cs >>= 1) {
-      if (cs > cap) continue;
-      cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3(cs);
-      cfg.blockDim = dim3(Shape<T, D, G>::W * 32);
-      cfg.dynamicSmemBytes = sm;
-      cudaLaunchAttribute at[1];
-      at[0].id = cudaLaunchAttributeClusterDimension;
-      at[0].val.clusterDim.x = cs;
-      at[0].val.clusterDim.y = 1;
-      at[0].val.clusterDim.z = 1;
-      cfg.attrs = at;
-      cfg.numAttrs = 1;
-      int ncl = 0;
-      if (cudaOccupancyMaxActiveClusters(&ncl, kc, &cfg) == cudaSuccess && ncl > 0) {
-        ctx->local_cluster_max = cs;
-        break;
-      }
-      cudaGetLastError();
-    }
+    int c0 = 0, c1 = 0;
+    ctx->local_cluster_max =
+        cluster_setup<T, D, G, Shape<T, D, G>::W, Shape<T, D, G>::NS>(ctx, c0);
+    ctx->local_wide_cluster_max = cluster_setup<T, D, G, ShapeWide::W, ShapeWide::NS>(ctx, c1);
+    ctx->local_wide_ctas = c1;
   }
   return ODA_OK;
 }
 
-template <typename T, int D, int G>
+template <typename T, int D, int G, int W, int NS>
 oda_status launch_cluster(oda_ctx* ctx, const AttnArgs& a, int grid, int cs, cudaStream_t st) {
-  auto k = kernel_ptr<T, D, G, true, true>();
-  const size_t sm = smem_bytes<T, D, G, true>(ctx->cfg.max_batch);
+  auto k = attn_kernel<T, D, G, W, NS, true, true>;
+  const size_t sm = smem_bytes_wn<T, D, G, W, NS>(ctx->cfg.max_batch);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(Shape<T, D, G>::W * 32);
+  cfg.blockDim = dim3(W * 32);
   cfg.dynamicSmemBytes = sm;
   cfg.stream = st;
   cudaLaunchAttribute at[2];
@@ -1165,7 +1195,12 @@ struct Launch {
       while (cs >= 2 && S * cs > ctx->attn_ctas_local) cs >>= 1;
       if (cs >= 2) {
         b.cluster = cs;
-        return launch_cluster<T, D, G>(ctx, b, S * cs, cs, st);
+        // one tile per warp even for a full ring: the wide shape
+        if (cs <= ctx->local_wide_cluster_max && S * cs <= ctx->local_wide_ctas &&
+            (b.ring_blocks + cs - 1) / cs <= ShapeWide::W)
+          return launch_cluster<T, D, G, ShapeWide::W, ShapeWide::NS>(ctx, b, S * cs, cs, st);
+        return launch_cluster<T, D, G, Shape<T, D, G>::W, Shape<T, D, G>::NS>(ctx, b, S * cs, cs,
+                                                                             st);
       }
     }
     return launch_one<T, D, G, RING>(ctx, b, RING ? ctx->attn_ctas_local : ctx->attn_ctas_full,

@@ -28,6 +28,8 @@ struct oda_ctx {
   int recall_parts_cap;      // capacity of recall_partials in floats
   int* plan_local;           // partition shared by a step's Local launches
   int local_cluster_max;     // largest cluster for the cluster-merge Local kernel (0: none)
+  int local_wide_cluster_max;  // the same for its one-tile-per-warp shape
+  int local_wide_ctas;       // CTAs of that shape one wave holds
 };
 
 namespace oda {
