@@ -328,21 +328,15 @@ attn_kernel(const AttnArgs a) {
 
   if (warp == 0) {
     if (CL) {
-      // cluster mode: segment = cluster, tiles split evenly over its ranks
+      // cluster mode: segment = cluster; the ranks split the whole ring
+      // evenly, whatever t is (tiles past the valid slots are masked), so the
+      // first copies need no global load; t itself is read by the consumer
       if (lane == 0) {
         const int cs = a.cluster;
         const int sg = (int)blockIdx.x / cs, rank = (int)blockIdx.x % cs;
-        const int b = sg / a.hkv, g = sg % a.hkv;
-        const bool okb = b < a.B;
-        const int t = okb ? a.seq_lens[b] : 0;
-        int nt = 0;
-        if (t < 1 || !okb) {
-          if (blockIdx.x == 0) record_error(a.err, ODA_ERR_BOUNDS);
-        } else {
-          nt = (a.sink + min(t, a.window) + ODA_TILE - 1) / ODA_TILE;
-        }
-        rowb[0] = okb ? b : 0;
-        rowt[0] = t;
+        const int g = sg % a.hkv;
+        const int nt = a.ring_blocks;
+        rowb[0] = sg / a.hkv;                    // < B: the grid is B * hkv * cs
         rowstart[0] = 0;
         rowstart[1] = nt * a.hkv;
         sinfo[0] = 1; sinfo[1] = nt * a.hkv; sinfo[2] = (int)gridDim.x; sinfo[3] = 1;
@@ -492,7 +486,16 @@ attn_kernel(const AttnArgs a) {
   locate(rowstart, nrows, a.hkv, lo, seg);
   while (true) {
     const int b = rowb[seg.i];
-    const int t = rowt[seg.i];
+    int t;
+    if (CL) {
+      t = a.seq_lens[b];                         // lands while the first copies fly
+      if (t < 1) {
+        if (tid == 0 && (int)blockIdx.x % a.cluster == 0) record_error(a.err, ODA_ERR_BOUNDS);
+        t = 0;                                   // every slot masked: an empty state
+      }
+    } else {
+      t = rowt[seg.i];
+    }
     const int s0 = seg.s1 - seg.nt;
 
     // this lane's DPL dims of the G query heads (exact, unscaled)
