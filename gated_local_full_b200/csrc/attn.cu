@@ -204,9 +204,8 @@ attn_kernel(const AttnArgs a) {
   int* sinfo = sflag + 4;                                          // [16] partition of this CTA
   int* stile = sinfo + 16;                                         // [W][NS] tile of each stage
   unsigned char* badst = reinterpret_cast<unsigned char*>(stile + W * NS);  // [W][NS]
-  float* cst = reinterpret_cast<float*>(
-      (reinterpret_cast<uintptr_t>(badst + W * NS) + 15) & ~uintptr_t(15));  // CL: [G][D+2]
-  float* racc = cst + G * (D + 2);             // CL: [cs][G*D/cs] pushed accumulators
+  float* racc = reinterpret_cast<float*>(
+      (reinterpret_cast<uintptr_t>(badst + W * NS) + 15) & ~uintptr_t(15));  // CL: [cs][G*D/cs]
   float* rml = racc + G * D;                   // CL: [16][G] pushed (m, l) pairs
 
   const int tid = threadIdx.x;
@@ -356,12 +355,47 @@ attn_kernel(const AttnArgs a) {
   int lo = sinfo[4], hi = sinfo[5];
   const int pbase_al = sinfo[6], nparts_al = sinfo[7], part_al = sinfo[8], vcta = sinfo[9];
   const int cta = (int)blockIdx.x;
+  // Cluster mode: each rank owns G*D/cs output elements of the segment. A
+  // rank merges its warps' states (or takes an empty one) and pushes, with
+  // remote shared-memory stores, its accumulator for every element to the
+  // element's owner and each head's (m, l) to every rank. The barrier that
+  // every rank arrived at on entry is waited for first, so every target CTA
+  // has started.
+  auto cluster_push = [&](bool filled) {
+    if constexpr (CL) {
+      namespace cg = cooperative_groups;
+      cg::cluster_group cl = cg::this_cluster();
+      const int cs = a.cluster;
+      const int rank = (int)cl.block_rank();
+      const int per = (G * D) / cs;
+      cluster_wait();
+      for (int o = tid; o < G * D; o += W * 32) {
+        const int h = o / D, dd = o % D;
+        float mt = -INFINITY, lt = 0.f, at = 0.f;
+        if (filled) {
+          for (int w2 = 0; w2 < W; ++w2) mt = fmaxf(mt, wstate[(w2 * G + h) * (D + 2) + D]);
+          if (mt != -INFINITY) {
+            for (int w2 = 0; w2 < W; ++w2) {
+              const float* st = wstate + (w2 * G + h) * (D + 2);
+              if (st[D] == -INFINITY) continue;
+              const float sc2 = fast_exp2(st[D] - mt);
+              lt += st[D + 1] * sc2;
+              at += st[dd] * sc2;
+            }
+          }
+        }
+        cl.map_shared_rank(racc, o / per)[rank * per + o % per] = at;
+        if (dd < cs)
+          reinterpret_cast<float2*>(cl.map_shared_rank(rml, dd))[rank * G + h] =
+              make_float2(mt, lt);
+      }
+    }
+  };
   // (cluster mode never leaves early: every CTA takes part in the merge)
   const bool has_work = nrows > 0 && total > 0 && lo < hi;
   if (!CL && !has_work) return;
   if (CL && !has_work) {
-    for (int i = tid; i < G * (D + 2); i += W * 32)
-      cst[i] = (i % (D + 2)) == D ? -INFINITY : 0.f;   // empty state: m = -inf, l = acc = 0
+    cluster_push(false);                         // an empty state: m = -inf, l = acc = 0
   } else {
 
   // K/V is read once per launch: stream it through L2 (the ring too, so no
@@ -719,25 +753,10 @@ attn_kernel(const AttnArgs a) {
     __syncthreads();
 
     if constexpr (CL) {
-      // cluster mode: this CTA's merged state goes to shared memory, where
-      // cluster rank 0 reads it (one segment per CTA, so the loop ends here)
-      for (int o = tid; o < G * D; o += W * 32) {
-        const int h = o / D, dd = o % D;
-        float mt = -INFINITY;
-        for (int w2 = 0; w2 < W; ++w2) mt = fmaxf(mt, wstate[(w2 * G + h) * (D + 2) + D]);
-        float lt = 0.f, at = 0.f;
-        if (mt != -INFINITY) {
-          for (int w2 = 0; w2 < W; ++w2) {
-            const float* st = wstate + (w2 * G + h) * (D + 2);
-            if (st[D] == -INFINITY) continue;
-            const float sc2 = fast_exp2(st[D] - mt);
-            lt += st[D + 1] * sc2;
-            at += st[dd] * sc2;
-          }
-        }
-        cst[h * (D + 2) + dd] = at;
-        if (dd == 0) { cst[h * (D + 2) + D] = mt; cst[h * (D + 2) + D + 1] = lt; }
-      }
+      // cluster mode (one segment per CTA, so the loop ends here): merge the
+      // warps and push each output element's accumulator straight to the
+      // rank that owns it, and each head's (m, l) to every rank
+      cluster_push(true);
       break;
     }
 
@@ -960,30 +979,13 @@ attn_kernel(const AttnArgs a) {
   }  // has_work
 
   if constexpr (CL) {
-    // Merge of the cluster's split KV. Each rank owns G*D/cs output elements;
-    // every rank pushes its accumulators for them, and its (m, l) per head,
-    // into the owner's shared memory (remote stores only), one cluster
-    // barrier publishes the stores, and each owner combines its elements
-    // from its own shared memory. No rank reads another rank's memory after
-    // that barrier, so ranks may exit as soon as they are done.
+    // Merge of the cluster's split KV (the pushes are in cluster_push).
     namespace cg = cooperative_groups;
     cg::cluster_group cl = cg::this_cluster();
     constexpr int GD = G * D;
     const int cs = a.cluster;
     const int rank = (int)cl.block_rank();
     const int per = GD / cs;
-    __syncthreads();                             // this CTA's state in cst is complete
-    cluster_wait();                              // every rank has started (arrived at entry)
-    for (int i = tid; i < GD; i += W * 32) {
-      const int h = i / D, dd = i % D;
-      float* dst = cl.map_shared_rank(racc, i / per);
-      dst[rank * per + i % per] = cst[h * (D + 2) + dd];
-    }
-    for (int j = tid; j < cs * G; j += W * 32) {
-      const int r2 = j / G, h = j % G;
-      float2* dst = reinterpret_cast<float2*>(cl.map_shared_rank(rml, r2));
-      dst[rank * G + h] = make_float2(cst[h * (D + 2) + D], cst[h * (D + 2) + D + 1]);
-    }
     cluster_arrive();                            // release: the pushes above
     cluster_wait();                              // acquire: every rank's pushes
     const int b = rowb[0], g = ((int)blockIdx.x / cs) % a.hkv;
@@ -1045,7 +1047,7 @@ size_t smem_bytes_wn(int max_batch) {
   s += 16 + 64;
   s += (size_t)W * NS * 4;
   s += (size_t)W * NS;
-  s += 16 + (size_t)(G * (D + 2) + G * D + 32 * G) * 4;   // cluster mode: state, merge buffers
+  s += 16 + (size_t)(G * D + 32 * G) * 4;     // cluster mode: pushed accumulators, (m, l)
   return (s + 127) & ~(size_t)127;
 }
 

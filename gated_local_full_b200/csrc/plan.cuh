@@ -44,6 +44,11 @@ __device__ __forceinline__ PlanHead plan_rows(const PlanIn& p, int* rowb, int* r
                                               int* rowstart, int* rowcs) {
   const int lane = threadIdx.x & 31;
   const bool ring = p.count == nullptr;
+  // with B <= 32 every lane loads one row's length and one compacted id
+  // before the count, so the three loads travel together instead of chaining
+  const bool small = p.B <= 32;
+  const int tl = (small && lane < p.B) ? __ldcg(p.seq_lens + lane) : 0;
+  const int il = (small && !ring && lane < p.B) ? __ldcg(p.idx + lane) : 0;
   int nr;
   if (ring) {
     nr = p.B;
@@ -58,14 +63,11 @@ __device__ __forceinline__ PlanHead plan_rows(const PlanIn& p, int* rowb, int* r
   for (int base = 0; base < nr; base += 32) {
     const int i = base + lane;
     int nt = 0;
-    // with B <= 32 every lane loads one row's length alongside the index,
-    // so the two loads overlap instead of chaining (all lanes shuffle)
-    const int tl = (p.B <= 32 && lane < p.B) ? __ldcg(p.seq_lens + lane) : 0;
-    const int bl = i < nr ? (ring ? i : __ldcg(p.idx + i)) : 0;
+    const int bl = i < nr ? (ring ? i : (small ? il : __ldcg(p.idx + i))) : 0;
     const bool okl = bl >= 0 && bl < p.B;
-    const int ts = __shfl_sync(0xffffffffu, tl, okl ? (bl & 31) : 0);
+    const int ts = __shfl_sync(0xffffffffu, tl, okl ? (bl & 31) : 0);   // all lanes shuffle
     if (i < nr) {
-      const int t = !okl ? 0 : (p.B <= 32 ? ts : __ldcg(p.seq_lens + bl));
+      const int t = !okl ? 0 : (small ? ts : __ldcg(p.seq_lens + bl));
       if (!okl || t < 1) {
         if (p.report) record_error(p.err, ODA_ERR_BOUNDS);
       } else if (ring) {
