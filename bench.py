@@ -53,6 +53,14 @@ def parse():
     ap.add_argument("--launch", choices=["graph", "plain"], default="graph",
                     help="graph: captured step with the IF node; plain: the same kernels "
                          "launched one by one (visible to ncu)")
+    ap.add_argument("--context", type=int, default=131072,
+                    help="context length t at the first step (the headline is 131072)")
+    ap.add_argument("--rate", type=float, default=0.125,
+                    help="Full-call rate: Bernoulli per step (the headline is 0.125)")
+    ap.add_argument("--mode", choices=["oda", "full-only"], default="oda",
+                    help="full-only: every step appends and runs Full attention in every "
+                         "layer, no Local, recall head or gate (dense decode, for the "
+                         "speedup and the short-context crossover)")
     return ap.parse_args()
 
 
@@ -335,7 +343,8 @@ def run_reference(args, rank, ws):
     if rank != 0:
         return
     import synth
-    w = synth.ctx128k(steps=args.warmup + args.steps, layers=args.layers)
+    w = synth.ctx128k(steps=args.warmup + args.steps, layers=args.layers, context=args.context,
+                      rate=args.rate)
     w.recall = True
     flags = w.flags()[:, 0]
     t_max = int(w.t0[0]) + w.steps
@@ -362,14 +371,20 @@ def run_reference(args, rank, ws):
 
 
 def config_block(w, args, ws):
-    return {"workload": "ctx128k_b1_l28: batch 1, 28 layers, 16/8 heads, d=128, bf16, "
-                        "t=131072+step, s=4, w=2048, Full calls Bernoulli(0.125) per step, "
-                        "recall head 6144->4096->1",
+    mode = getattr(args, "mode", "oda")
+    desc = (f"{w.name}: batch 1, {w.layers} layers, 16/8 heads, d=128, bf16, "
+            f"t={int(w.t0[0])}+step, s=4, w=2048, ")
+    desc += ("Full calls Bernoulli(%g) per step, recall head 6144->4096->1" % w.flag_rate
+             if mode == "oda" else "dense decode: append + Full attention every layer, every step")
+    return {"workload": desc, "mode": mode,
             "batch_per_gpu": int(w.batch), "global_batch": int(w.batch * ws),
             "context": int(w.t0[0]), "layers": int(w.layers), "hq": w.hq, "hkv": w.hkv,
-            "head_dim": w.d, "sink": w.sink, "window": w.window, "full_call_rate": 0.125,
+            "head_dim": w.d, "sink": w.sink, "window": w.window,
+            "full_call_rate": w.flag_rate if mode == "oda" else 1.0,
             "parallelism": f"replicas x{ws}", "launch": getattr(args, "launch", "graph"),
-            "l2": "no flush needed: per-step reads (ring 235 MB, Full 15 GB) exceed the 126 MB L2"}
+            "l2": "no flush needed: per-step reads (ring %d MB, Full %d GB) exceed the 126 MB L2"
+                  % (round(w.layers * min(int(w.t0[0]), w.sink + w.window) * KV_BYTES_PER_TOKEN_LAYER / 1e6),
+                     round(w.layers * int(w.t0[0]) * KV_BYTES_PER_TOKEN_LAYER / 1e9))}
 
 
 # ----------------------------------------------------------------------------
@@ -386,7 +401,7 @@ def run_oda(args, rank, ws, local):
 
     torch.cuda.set_device(local)
     K, W = args.steps, args.warmup
-    w = synth.ctx128k(steps=W + K, layers=args.layers)
+    w = synth.ctx128k(steps=W + K, layers=args.layers, context=args.context, rate=args.rate)
     w.recall = True                                   # recall head runs every step
     flags = w.flags()[:, 0]
     bt, nb = w.paging()
@@ -411,10 +426,34 @@ def run_oda(args, rank, ws, local):
     assert ctx.get_device_error() == 0
     stream = torch.cuda.current_stream()
 
+    dense = args.mode == "full-only"
+    if dense:
+        # dense decode on the same kernels: commit the token, then Full
+        # attention for every row in every layer, captured once as a graph
+        cnt_all = torch.full((1,), w.batch, dtype=torch.int32, device="cuda")
+        idx_all = torch.arange(w.batch, dtype=torch.int32, device="cuda")
+
+        def dense_step():
+            ctx.append_kv(0, w.layers, st.k_new, st.v_new, st.seq_lens, dw.block_table, dw.cache,
+                          dw.ring, w.batch)
+            for l in range(w.layers):
+                ctx.full_attn_gated(l, st.q[l], st.seq_lens, dw.block_table, dw.cache, idx_all,
+                                    cnt_all, st.out[l], None, w.batch)
+
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        dgraph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(dgraph, stream=side):
+            dense_step()
+        stream.wait_stream(side)
+        run_step = dgraph.replay
+    else:
+        run_step = st.run
+
     sampler = ClockSampler(gpu_id(local))
     for i in range(W):
         st.feed_record(recs, i)
-        st.run()
+        run_step()
     torch.cuda.synchronize()
     barrier(ws)
     torch.cuda.synchronize()
@@ -423,7 +462,7 @@ def run_oda(args, rank, ws, local):
     e0.record(stream)
     for i in range(W, W + K):
         st.feed_record(recs, i)
-        st.run()
+        run_step()
     e1.record(stream)
     torch.cuda.synchronize()
     h1 = time.time()
@@ -434,10 +473,15 @@ def run_oda(args, rank, ws, local):
     t_max = max_over_ranks(elapsed, ws)
     timed = list(range(W, W + K))
     n_flag = int(flags[timed].sum())
-    kv_bytes = sum(step_kv_bytes(int(w.t0[0]) + i, bool(flags[i]), w.layers) for i in timed)
-    # append, Local x L, recall, gate, then Full x L: behind the IF node only
-    # flagged steps launch them; plain launches issue them every step
-    launches = K * (w.layers + 4) + (n_flag if args.launch == "graph" else K) * w.layers
+    if dense:
+        kv_bytes = sum(w.layers * (int(w.t0[0]) + i + 2) * KV_BYTES_PER_TOKEN_LAYER
+                       for i in timed)
+        launches = K * (w.layers + 1)
+    else:
+        kv_bytes = sum(step_kv_bytes(int(w.t0[0]) + i, bool(flags[i]), w.layers) for i in timed)
+        # append, Local x L, recall, gate, then Full x L: behind the IF node
+        # only flagged steps launch them; plain launches issue them every step
+        launches = K * (w.layers + 4) + (n_flag if args.launch == "graph" else K) * w.layers
 
     # ---- dominant kernel: Full attention. As in a flagged step, the L layers'
     # launches run back to back: the runs of up to 16 flagged steps are
@@ -489,7 +533,7 @@ def run_oda(args, rank, ws, local):
         a.record(stream)
         for j in range(n_e2e):
             st.feed_record(hrec, j)
-            st.run()
+            run_step()
             res.copy_(st.out[w.layers - 1], non_blocking=True)
             cnt.copy_(st.count, non_blocking=True)
             stream.synchronize()
@@ -503,7 +547,7 @@ def run_oda(args, rank, ws, local):
 
     sampler.stop()
     cpu = None
-    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline and not dense:
         steps = cpu_sample_steps(timed, flags, args.cpu_steps)
         sample = OracleSample(w, int(w.t0[0]) + S)
         secs = {i: sample.step_seconds(i, bool(flags[i])) for i in steps}
@@ -521,7 +565,8 @@ def run_oda(args, rank, ws, local):
             "data": "synthetic (seeded counter-based generator; no datasets or weights)",
             "config": config_block(w, args, ws),
             "kv_gbs": kv_gbs, "kv_frac_of_hbm": kv_gbs / hbm,
-            "kv_bytes_per_step": kv_bytes / K, "full_call_rate_realised": n_flag / K,
+            "kv_bytes_per_step": kv_bytes / K,
+            "full_call_rate_realised": 1.0 if dense else n_flag / K,
             "recall_weight_bytes_per_step": int(w.recall_hidden * 3 * w.hidden * 2),
             "roofline": {"bound": "hbm", "achieved": full_gbs, "peak": hbm, "unit": "GB/s",
                          "frac": full_gbs / hbm, "traffic": traffic,

@@ -312,13 +312,17 @@ def ctx16k(batch: int = 8) -> Workload:
     return w
 
 
-def ctx128k(steps: int = 1024, layers: int = 28) -> Workload:
+def ctx128k(steps: int = 1024, layers: int = 28, context: int = 131072,
+            rate: float = 0.125) -> Workload:
     """bf16, batch 1, 28 layers, 16/8 heads, d=128, t = 131072 at the first
-    step, 1024 decode steps, Full calls Bernoulli(0.125) per step."""
-    return Workload(name="ctx128k_b1_l28", dtype="bf16", layers=layers, batch=1, hq=16, hkv=8,
+    step, 1024 decode steps, Full calls Bernoulli(0.125) per step. `context`
+    and `rate` give the same request at another length or call rate."""
+    name = ("ctx128k_b1_l28" if (context, rate, layers) == (131072, 0.125, 28)
+            else f"ctx{context}_rho{rate:g}_b1_l{layers}")
+    return Workload(name=name, dtype="bf16", layers=layers, batch=1, hq=16, hkv=8,
                     d=128, sink=4, window=2048, block_size=16,
-                    t0=np.array([131072], np.int64), steps=steps, seed=2,
-                    flag_rate=0.125, flag_per="step")
+                    t0=np.array([context], np.int64), steps=steps, seed=2,
+                    flag_rate=rate, flag_per="step")
 
 
 MIXED_RATES = (0.0, 0.125, 0.41, 1.0)
