@@ -35,6 +35,12 @@
  *     skips the bad access and carries on, it never traps.
  *   - Element types: ODA_BF16 (storage bf16, arithmetic fp32) or ODA_F32.
  *     Queries, K/V, rings and outputs share the context's dtype.
+ *   - Kernels are launched with programmatic dependent launch: a kernel may
+ *     become resident while the previous one on the stream still runs, but
+ *     it reads no input and writes nothing before that kernel has completed
+ *     (griddepcontrol.wait), so stream order holds as for plain launches.
+ *     Before the wait it only warms L2 with bulk prefetches of the K/V it is
+ *     about to read, which read no values.
  */
 #ifndef ODA_H
 #define ODA_H
