@@ -37,10 +37,12 @@
  *     Queries, K/V, rings and outputs share the context's dtype.
  *   - Kernels are launched with programmatic dependent launch: a kernel may
  *     become resident while the previous one on the stream still runs, but
- *     it reads no input and writes nothing before that kernel has completed
- *     (griddepcontrol.wait), so stream order holds as for plain launches.
- *     Before the wait it only warms L2 with bulk prefetches of the K/V it is
- *     about to read, which read no values.
+ *     nothing it computes or writes depends on memory read before that kernel
+ *     has completed (griddepcontrol.wait), so stream order holds as for plain
+ *     launches. Before the wait an attention kernel may read row ids,
+ *     lengths and block-table entries (bypassing L1) only to choose which
+ *     K/V lines to warm in L2 with bulk prefetches; these are read again
+ *     after the wait, and a prefetch returns no value.
  */
 #ifndef ODA_H
 #define ODA_H
