@@ -424,6 +424,18 @@ attn_kernel(const AttnArgs a) {
     hi = seg_s0 + (int)(((long long)(part_al + 1) * pool0) / nparts_al);
   }
   const bool use_pool = pool0 < seg_nt;
+  // cluster mode has one segment per CTA: its queries and t are loaded
+  // before the first copies are issued, so they land while the copies fly
+  float2 qpre[G][DP2];
+  int tpre = 0;
+  if constexpr (CL) {
+    tpre = a.seq_lens[seg_b];
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+      Chunk<T>::load(reinterpret_cast<const T*>(a.q) +
+                         ((long long)seg_b * hq + prod.g * G + h) * D + li * DPL,
+                     qpre[h]);
+  }
   int q0 = seg_nt, q1 = seg_nt, qb0 = -1, qb1 = -1;   // lane 0: grabbed pool tiles, blocks
   auto grab = [&](int& q, int& qb) {                  // lane 0 only
     q = pool0 + atomicAdd(&a.dyn[sigma0], 1);
@@ -522,7 +534,7 @@ attn_kernel(const AttnArgs a) {
     const int b = rowb[seg.i];
     int t;
     if (CL) {
-      t = a.seq_lens[b];                         // lands while the first copies fly
+      t = tpre;                                  // loaded before the first copies
       if (t < 1) {
         if (tid == 0 && (int)blockIdx.x % a.cluster == 0) record_error(a.err, ODA_ERR_BOUNDS);
         t = 0;                                   // every slot masked: an empty state
@@ -536,9 +548,14 @@ attn_kernel(const AttnArgs a) {
     float2 q2[G][DP2];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
-      const T* qp = reinterpret_cast<const T*>(a.q) +
-                    ((long long)b * hq + seg.g * G + h) * D + li * DPL;
-      Chunk<T>::load(qp, q2[h]);
+      if constexpr (CL) {
+#pragma unroll
+        for (int e = 0; e < DP2; ++e) q2[h][e] = qpre[h][e];
+      } else {
+        const T* qp = reinterpret_cast<const T*>(a.q) +
+                      ((long long)b * hq + seg.g * G + h) * D + li * DPL;
+        Chunk<T>::load(qp, q2[h]);
+      }
     }
     float m_run[G], l_run[G];
     float2 acc[G][DP2];
