@@ -836,7 +836,7 @@ attn_kernel(const AttnArgs a) {
         // L2 round trip.
         constexpr int NCH = G * D / 4;                 // float4 chunks of the output
         constexpr int SPLIT = (W * 32) / NCH > 0 ? (W * 32) / NCH : 1;
-        constexpr int MAXB = G >= 4 ? 4 : 8;           // partial chunks held per thread
+        constexpr int MAXB = G >= 4 ? 4 : (G == 2 ? 16 : 8);   // partial chunks held per thread
         float* sml = wstate;                           // [nparts][G][2]
         float* ssc = sml + 2 * nparts * G;             // [nparts][G] scale factors
         float* stot = ssc + nparts * G;                // [2G]: m_tot, l_tot
