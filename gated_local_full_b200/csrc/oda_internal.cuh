@@ -26,6 +26,7 @@ struct oda_ctx {
   int* recall_tickets;       // recall-head split reduction counters
   float* recall_partials;    // recall-head split partials
   int recall_parts_cap;      // capacity of recall_partials in floats
+  int recall_cluster_max;    // largest cluster for the recall head's split-K (0: none)
   int* plan_local;           // partition shared by a step's Local launches
   int local_cluster_max;     // largest cluster for the cluster-merge Local kernel (0: none)
   int local_wide_cluster_max;  // the same for its one-tile-per-warp shape

@@ -24,6 +24,7 @@
 //     fixed order, adds b1, applies GELU and the w2 dot product; the last
 //     m-tile sums the per-tile dot products in order and adds b2. The result
 //     is deterministic run to run.
+#include <cooperative_groups.h>
 #include <cuda.h>
 
 #include "oda_internal.cuh"
@@ -405,6 +406,217 @@ recall_kernel(const __grid_constant__ CUtensorMap tm_w1, const __grid_constant__
   }
 }
 
+// Split-K over a thread-block cluster. For the common shape (hidden / 128
+// m-tiles times KS fit the SMs, batch <= 64) the K range of each m-tile is
+// split evenly over a cluster of KS CTAs instead of the stream-K order above:
+// no CTA spans two m-tiles, and the split is reduced in distributed shared
+// memory. Rank r owns rows [r*128/KS, (r+1)*128/KS) of the m-tile: every rank
+// pushes its accumulator rows to their owners with remote stores, one cluster
+// barrier publishes them, each owner sums its rows' KS parts in rank order,
+// adds b1, applies GELU and w2 and reduces over its rows, and writes one
+// partial dot product per batch row; the last CTA of the grid (ticket) sums
+// those in a fixed order and adds b2. Deterministic, like the stream-K path.
+constexpr int CL_MAX_N = 64;                             // batch rows (16, 32 or 64 columns)
+
+__global__ void __launch_bounds__(192, 1)
+recall_cluster_kernel(const __grid_constant__ CUtensorMap tm_w1,
+                      const __grid_constant__ CUtensorMap tm_x0,
+                      const __grid_constant__ CUtensorMap tm_x1,
+                      const __grid_constant__ CUtensorMap tm_x2, const RecallArgs a, int KS) {
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw = smem_addr(smem_raw);
+  const uint32_t pad = ((raw + 1023u) & ~1023u) - raw;
+  unsigned char* smem = smem_raw + pad;
+  const int S = a.stages;
+  const int N = a.N;
+  const uint32_t b_stage_bytes = (uint32_t)N * BK * 2;
+  unsigned char* sa = smem;
+  unsigned char* sb = sa + (size_t)S * A_STAGE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sb + (size_t)S * b_stage_bytes);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + S;
+  uint64_t* acc_full = bars + 2 * S;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+  int* sflag = reinterpret_cast<int*>(tmem_slot + 1);
+  float* rbuf = reinterpret_cast<float*>(
+      (reinterpret_cast<uintptr_t>(sflag + 4) + 15) & ~uintptr_t(15));   // [KS][128/KS][N]
+  float* red = rbuf + BM * N;                             // [192] partial sums
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int rank = (int)blockIdx.x % KS;
+  const int mt = (int)blockIdx.x / KS;
+  const int kb0 = (rank * a.KB) / KS, kb1 = ((rank + 1) * a.KB) / KS;
+  const int RP = BM / KS;                                 // rows each rank owns
+  uint32_t ncols = 32;
+  while ((int)ncols < N) ncols <<= 1;
+
+  cluster_arrive_relaxed();                               // "started": waited for before any push
+  if (tid == 0) {
+    for (int s2 = 0; s2 < S; ++s2) {
+      mbar_init(smem_addr(&full[s2]), 1);
+      mbar_init(smem_addr(&empty[s2]), 1);
+    }
+    mbar_init(smem_addr(acc_full), 1);
+    fence_mbar_init();
+  }
+  pdl_wait();
+  pdl_launch_dependents();
+  if (warp == 0) {
+    __syncwarp();
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_addr(tmem_slot)),
+                 "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const uint32_t tx = A_STAGE_BYTES + b_stage_bytes;
+      for (int kb = kb0, i = 0; kb < kb1; ++kb, ++i) {
+        const int s2 = i % S;
+        const uint32_t par = (uint32_t)(((i / S) & 1) ^ 1);
+        if (!mbar_wait_bounded(smem_addr(&empty[s2]), par, kWaitLimitNs)) {
+          record_error(a.err, ODA_ERR_TIMEOUT);
+          break;
+        }
+        const uint32_t fb = smem_addr(&full[s2]);
+        mbar_arrive_expect_tx(fb, tx);
+        tma_load_2d(smem_addr(sa + (size_t)s2 * A_STAGE_BYTES), &tm_w1, kb * BK, mt * BM, fb);
+        const int kglob = kb * BK;
+        const int seg = kglob / a.H;
+        const int kin = kglob - seg * a.H;
+        const CUtensorMap* xm = seg == 0 ? &tm_x0 : (seg == 1 ? &tm_x1 : &tm_x2);
+        tma_load_2d(smem_addr(sb + (size_t)s2 * b_stage_bytes), xm, kin, 0, fb);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = umma_idesc_bf16(N);
+      for (int kb = kb0, i = 0; kb < kb1; ++kb, ++i) {
+        const int s2 = i % S;
+        if (!mbar_wait_bounded(smem_addr(&full[s2]), (uint32_t)((i / S) & 1), kWaitLimitNs)) {
+          record_error(a.err, ODA_ERR_TIMEOUT);
+          break;
+        }
+        fence_after_sync();
+        const uint64_t ad = umma_desc_sw128(smem_addr(sa + (size_t)s2 * A_STAGE_BYTES));
+        const uint64_t bd = umma_desc_sw128(smem_addr(sb + (size_t)s2 * b_stage_bytes));
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk)
+          umma_bf16(tmem, ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), idesc,
+                    (kb == kb0 && kk == 0) ? 0u : 1u);
+        umma_commit(smem_addr(&empty[s2]));
+      }
+      umma_commit(smem_addr(acc_full));                   // after every MMA above
+    }
+  }
+
+  // ------------------------------------------------- push rows to owners
+  namespace cg = cooperative_groups;
+  cg::cluster_group cl = cg::this_cluster();
+  if (tid == 64) {
+    const bool got = kb0 < kb1 &&
+                     mbar_wait_bounded(smem_addr(acc_full), 0u, kWaitLimitNs);
+    if (!got && kb0 < kb1) record_error(a.err, ODA_ERR_TIMEOUT);
+    sflag[0] = got ? 1 : 0;
+  }
+  __syncthreads();
+  fence_after_sync();
+  cluster_wait();                                         // every rank has started
+  if (warp >= 2) {
+    const int q = warp & 3;                               // TMEM lane quarter of this warp
+    const int m = q * 32 + lane;                          // row of the m-tile
+    const int owner = m / RP;
+    float* dst = cl.map_shared_rank(rbuf, owner) + ((size_t)rank * RP + (m - owner * RP)) * N;
+    for (int n0 = 0; n0 < N; n0 += 16) {
+      float v[16];
+      if (sflag[0]) {
+        tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)n0, v);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) v[e] = 0.f;
+      }
+#pragma unroll
+      for (int e = 0; e < 16; e += 4)
+        *reinterpret_cast<float4*>(dst + n0 + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+    }
+  }
+  fence_before_sync();
+  cluster_arrive();                                       // release: the pushes
+  cluster_wait();                                         // acquire: every rank's pushes
+
+  // ------------------------------------- owner: b1, GELU, w2 over its rows
+  if (warp >= 2) {
+    const int j = tid - 64;                               // 0..127
+    const int TPN = BM / N;                               // threads per batch row
+    const int n = j % N, t0 = j / N;
+    float s = 0.f;
+    for (int rl = t0; rl < RP; rl += TPN) {               // fixed order
+      float u = 0.f;
+      for (int r2 = 0; r2 < KS; ++r2) u += rbuf[((size_t)r2 * RP + rl) * N + n];
+      const int row = mt * BM + rank * RP + rl;
+      s += a.w2[row] * gelu_erf(u + a.b1[row]);
+    }
+    red[j] = s;
+  }
+  __syncthreads();
+  if (warp >= 2) {
+    const int j = tid - 64;
+    const int TPN = BM / N;
+    if (j < N) {
+      float s = 0.f;
+      for (int t2 = 0; t2 < TPN; ++t2) s += red[t2 * N + j];
+      a.spart[(size_t)blockIdx.x * N + j] = s;
+    }
+  }
+  __syncthreads();
+  if (tid == 64) {
+    __threadfence();
+    const int prev = atomicAdd(&a.tickets[MAX_MT], 1);
+    sflag[1] = (prev == (int)gridDim.x - 1) ? 1 : 0;
+  }
+  __syncthreads();
+  if (sflag[1]) {
+    __threadfence();
+    // every CTA's partial loaded at once: thread (grp, n) sums CTAs
+    // grp, grp + ngrp, ... of batch row n; the groups are then added in order
+    const int ngrp = 192 / a.B;                           // B <= 64: at least 3 groups
+    const int n = tid % a.B, grp = tid / a.B;
+    float v = 0.f;
+    if (grp < ngrp) {
+      for (int c2 = grp; c2 < (int)gridDim.x; c2 += ngrp) v += __ldcg(a.spart + (size_t)c2 * N + n);
+      red[grp * a.B + n] = v;
+    }
+    __syncthreads();
+    if (tid < a.B) {
+      float t2 = 0.f;
+      for (int g2 = 0; g2 < ngrp; ++g2) t2 += red[g2 * a.B + tid];
+      a.scores[tid] = t2 + a.b2;
+    }
+    if (tid == 0) a.tickets[MAX_MT] = 0;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    __syncwarp();
+    // every MMA must have completed before TMEM is released
+    if (kb0 < kb1 && !mbar_wait_bounded(smem_addr(acc_full), 0u, kWaitLimitNs) && lane == 0)
+      record_error(a.err, ODA_ERR_TIMEOUT);
+    __syncwarp();
+    fence_after_sync();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(ncols)
+                 : "memory");
+  }
+}
+
 // ------------------------------------------------------------ host side
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -451,6 +663,20 @@ size_t smem_for(int n, int s) {
          4 * MAX_N * 4 + 64;
 }
 
+// Stages and shared memory of the cluster kernel (its row buffer comes first).
+int cl_stages_for(int n) {
+  const int per = A_STAGE_BYTES + n * BK * 2;
+  int s = (200 * 1024 - BM * n * 4) / per;
+  if (s > 8) s = 8;
+  if (s < 2) s = 2;
+  return s;
+}
+
+size_t cl_smem_for(int n, int s) {
+  return 1024 + (size_t)s * (A_STAGE_BYTES + n * BK * 2) + (size_t)(2 * s + 1) * 8 + 4 + 16 + 16 +
+         (size_t)(BM * n + 192) * 4 + 64;
+}
+
 }  // namespace
 
 namespace oda_impl {
@@ -466,6 +692,32 @@ oda_status recall_setup(oda_ctx* ctx) {
   ctx->recall_parts_cap = (int)((size_t)(ctx->num_sms + MAX_MT) * MAX_N * BM);
   ODA_CUDA_TRY(cudaMalloc(&ctx->recall_tickets, (MAX_MT + 1) * sizeof(int)));
   ODA_CUDA_TRY(cudaMemset(ctx->recall_tickets, 0, (MAX_MT + 1) * sizeof(int)));
+  // the cluster split-K kernel: the largest cluster (8, 4, 2) the GPU holds
+  ctx->recall_cluster_max = 0;
+  const size_t csm = cl_smem_for(CL_MAX_N, cl_stages_for(CL_MAX_N));
+  if (cudaFuncSetAttribute(recall_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)csm) == cudaSuccess) {
+    for (int ks = 8; ks >= 2; ks >>= 1) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(ks);
+      cfg.blockDim = dim3(192);
+      cfg.dynamicSmemBytes = csm;
+      cudaLaunchAttribute at[1];
+      at[0].id = cudaLaunchAttributeClusterDimension;
+      at[0].val.clusterDim.x = ks;
+      at[0].val.clusterDim.y = 1;
+      at[0].val.clusterDim.z = 1;
+      cfg.attrs = at;
+      cfg.numAttrs = 1;
+      int ncl = 0;
+      if (cudaOccupancyMaxActiveClusters(&ncl, recall_cluster_kernel, &cfg) == cudaSuccess &&
+          ncl > 0) {
+        ctx->recall_cluster_max = ks;
+        break;
+      }
+    }
+  }
+  cudaGetLastError();
   return ODA_OK;
 }
 
@@ -496,6 +748,32 @@ oda_status launch_recall(oda_ctx* ctx, const void* h_prev, const void* emb, cons
   a.MT = hidden / BM;
   a.KB = (int)(K / BK);
   a.H = H;
+  // cluster split-K when every m-tile gets a whole cluster within one wave
+  int KS = 0;
+  if (N == 16 || N == 32 || N == 64) {
+    for (int ks = ctx->recall_cluster_max; ks >= 2; ks >>= 1)
+      if (a.MT * ks <= ctx->num_sms && a.KB >= ks) { KS = ks; break; }
+  }
+  if (KS >= 2) {
+    a.stages = cl_stages_for(N);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.MT * KS);
+    cfg.blockDim = dim3(192);
+    cfg.dynamicSmemBytes = cl_smem_for(N, a.stages);
+    cfg.stream = st;
+    cudaLaunchAttribute at[2];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = KS;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, recall_cluster_kernel, tw, t0, t1, t2, a, KS) == cudaSuccess
+               ? ODA_OK
+               : ODA_ERR_CUDA;
+  }
   a.stages = stages_for(N);
   const int U = a.MT * a.KB;
   const int grid = U < ctx->num_sms ? U : ctx->num_sms;
