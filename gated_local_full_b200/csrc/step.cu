@@ -180,6 +180,20 @@ oda_status oda_step_graph_launch(oda_graph* g, oda_stream stream) {
   return ODA_OK;
 }
 
+oda_status oda_step_graph_run_io(oda_graph* g, const void* h_in, void* d_in, size_t in_bytes,
+                                 const void* d_out, void* h_out, size_t out_bytes,
+                                 oda_stream stream) {
+  if (!g || !g->exec) return ODA_ERR_ARG;
+  if ((in_bytes && (!h_in || !d_in)) || (out_bytes && (!d_out || !h_out))) return ODA_ERR_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (in_bytes) ODA_CUDA_TRY(cudaMemcpyAsync(d_in, h_in, in_bytes, cudaMemcpyHostToDevice, st));
+  ODA_CUDA_TRY(cudaGraphLaunch(g->exec, st));
+  if (out_bytes)
+    ODA_CUDA_TRY(cudaMemcpyAsync(h_out, d_out, out_bytes, cudaMemcpyDeviceToHost, st));
+  ODA_CUDA_TRY(cudaStreamSynchronize(st));
+  return ODA_OK;
+}
+
 oda_status oda_step_graph_destroy(oda_graph* g) {
   if (!g) return ODA_OK;
   if (g->exec) cudaGraphExecDestroy(g->exec);

@@ -30,7 +30,8 @@ EXPORTS = (
     "oda_layout", "oda_create", "oda_destroy", "oda_append_kv", "oda_ring_init",
     "oda_local_attn", "oda_recall_score", "oda_gate", "oda_full_attn_gated",
     "oda_get_device_error", "oda_selftest_wait_timeout", "oda_step_run",
-    "oda_step_graph_create", "oda_step_graph_launch", "oda_step_graph_destroy", "oda_version",
+    "oda_step_graph_create", "oda_step_graph_launch", "oda_step_graph_run_io",
+    "oda_step_graph_destroy", "oda_version",
     "oda_full_attn_gated_static",
 )
 
@@ -92,6 +93,7 @@ def lib() -> ctypes.CDLL:
         "oda_step_run": [vp, POINTER(OdaStepDesc), vp],
         "oda_step_graph_create": [vp, POINTER(OdaStepDesc), POINTER(c_void_p)],
         "oda_step_graph_launch": [vp, vp],
+        "oda_step_graph_run_io": [vp, vp, vp, ctypes.c_size_t, vp, vp, ctypes.c_size_t, vp],
         "oda_step_graph_destroy": [vp],
         "oda_full_attn_gated_static": [POINTER(OdaConfig), c_int, vp, vp, vp, vp, vp, vp, vp,
                                        vp, c_int, vp, vp],
@@ -119,6 +121,17 @@ def ptr(x) -> Optional[int]:
         return x
     if not x.is_cuda:
         raise ValueError("tensor must live on the GPU")
+    if not x.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return x.data_ptr()
+
+
+def hptr(x) -> Optional[int]:
+    """Host pointer of a contiguous CPU tensor (pin it for asynchronous copies), or None."""
+    if x is None:
+        return None
+    if x.is_cuda:
+        raise ValueError("tensor must live in host memory")
     if not x.is_contiguous():
         raise ValueError("tensor must be contiguous")
     return x.data_ptr()
@@ -158,6 +171,14 @@ class OdaGraph:
 
     def launch(self, stream=None) -> None:
         _check(lib().oda_step_graph_launch(self.handle, _stream(stream)), "oda_step_graph_launch")
+
+    def run_io(self, h_in, d_in, d_out, h_out, stream=None) -> None:
+        """Copy h_in -> d_in, launch, copy d_out -> h_out, wait (one call)."""
+        nin = h_in.numel() * h_in.element_size() if h_in is not None else 0
+        nout = h_out.numel() * h_out.element_size() if h_out is not None else 0
+        _check(lib().oda_step_graph_run_io(self.handle, hptr(h_in), ptr(d_in), nin, ptr(d_out),
+                                           hptr(h_out), nout, _stream(stream)),
+               "oda_step_graph_run_io")
 
     def close(self) -> None:
         if self.handle:

@@ -58,13 +58,18 @@ class DecodeStep:
             setattr(self, name, self.record[o:o + nbytes].view(fdt).view(shape))
         if not external_scores:
             self.gate_scores = None
-        # ---- outputs
-        self.out = torch.zeros((L, B, hq, d), dtype=dt, device=dev)
+        # ---- outputs; the last layer's output and the count are contiguous
+        # (the "result" a host loop reads back every step, in one copy)
+        esz = torch.empty((), dtype=dt).element_size()
+        out_bytes = L * B * hq * d * esz
+        self._outbuf = torch.zeros(out_bytes + 16, dtype=torch.uint8, device=dev)
+        self.out = self._outbuf[:out_bytes].view(dt).view(L, B, hq, d)
+        self.count = self._outbuf[out_bytes:out_bytes + 4].view(torch.int32)
+        self.result = self._outbuf[(L - 1) * B * hq * d * esz:out_bytes + 4]
         self.lse = torch.zeros((L, B, hq), dtype=torch.float32, device=dev) if with_lse else None
         self.scores = torch.zeros(B, dtype=torch.float32, device=dev)
         self.flags = torch.zeros(B, dtype=torch.uint8, device=dev)
         self.idx = torch.zeros(B, dtype=torch.int32, device=dev)
-        self.count = torch.zeros(1, dtype=torch.int32, device=dev)
         self.kv_cache, self.ring, self.block_table = kv_cache, ring, block_table
         self.recall = recall
         rk = {}
@@ -120,6 +125,27 @@ class DecodeStep:
             self.graph.launch(stream)
         else:
             self.ctx.step_run(self.desc, stream)
+
+    def new_result(self):
+        """Pinned host buffer shaped like `result` (last layer's output, then the count)."""
+        import torch
+        return torch.empty(self.result.numel(), dtype=torch.uint8).pin_memory()
+
+    def run_io(self, h_record, h_result, stream=None) -> None:
+        """One host-driven step in one library call: the packed inputs from the
+        host record h_record (pinned, record_bytes), the captured step, and
+        the result back into h_result (see new_result); returns when h_result
+        holds it. Needs the captured graph."""
+        if self.graph is None:
+            raise RuntimeError("run_io needs the captured step graph")
+        self.graph.run_io(h_record, self.record, self.result, h_result, stream)
+
+    def split_result(self, h_result):
+        """(last layer's output, count) views of a result buffer."""
+        import torch
+        n = self.result.numel() - 4
+        out = h_result[:n].view(self.out.dtype).view(self.out.shape[1:])
+        return out, h_result[n:n + 4].view(torch.int32)
 
     def close(self) -> None:
         if self.graph is not None:

@@ -292,6 +292,18 @@ oda_status oda_step_run(oda_ctx* ctx, const oda_step_desc* d, oda_stream stream)
  * baked in: refill the same buffers between launches. */
 oda_status oda_step_graph_create(oda_ctx* ctx, const oda_step_desc* d, oda_graph** out);
 oda_status oda_step_graph_launch(oda_graph* g, oda_stream stream);
+
+/* One step of a host-driven decode loop in a single call: copy in_bytes from
+ * host memory h_in to device memory d_in (the step's packed inputs), launch
+ * the step graph, copy out_bytes from device memory d_out to host memory
+ * h_out (the step's results), then wait for the stream. Each copy is one
+ * cudaMemcpyAsync on `stream`; host buffers should be pinned for the copies
+ * to be asynchronous. in_bytes or out_bytes may be 0 (that copy is skipped).
+ * Returns after h_out holds the results; a CUDA error returns ODA_ERR_CUDA.
+ * Device-detected errors still go to the context's error word. */
+oda_status oda_step_graph_run_io(oda_graph* g, const void* h_in, void* d_in, size_t in_bytes,
+                                 const void* d_out, void* h_out, size_t out_bytes,
+                                 oda_stream stream);
 oda_status oda_step_graph_destroy(oda_graph* g);
 
 /* Library version string. */

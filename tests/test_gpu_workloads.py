@@ -130,3 +130,39 @@ def test_graph_equals_plain_launches_and_skips_full(torch):
             ref = hx.oracle_row(w, 1, l, b)
             want = ref["full"] if b % 2 == 0 else ref["local"]
             hx.assert_close(out[l, b], want, *hx.tol(w), what=f"graph l{l} b{b}")
+
+
+def test_run_io_matches_launch_and_copies(torch):
+    """oda_step_graph_run_io (host record in, step, result out, one call)
+    gives the same last-layer output and count as feeding the record,
+    launching the graph and copying back separately; and the result matches
+    the oracle (Full for the flagged rows, Local for the others)."""
+    from gated_local_full_b200.runtime import DecodeStep
+    w = synth.custom("runio", layers=2, batch=3, hq=8, hkv=4, t0=(700, 90, 1500),
+                     fixed_scores=(1.0, -1.0, 1.0), steps=2)
+    ctx, dw = hx.setup(w)
+    st = DecodeStep(ctx, 3, dw.cache, dw.ring, dw.block_table, external_scores=True)
+    recs = st.new_records(w.steps)
+    for i in range(w.steps):
+        st.pack(recs, i, q=dw.q[i], k_new=dw.k_new[i], v_new=dw.v_new[i],
+                seq_lens=dw.seq_lens[i], gate_scores=dw.scores[i])
+    hrec = st.new_records(w.steps, pin=True)
+    hrec.copy_(recs.cpu())
+    # step 0 the separate way, step 1 in one call
+    st.feed_record(recs, 0)
+    st.run()
+    hres = st.new_result()
+    st.run_io(hrec[1], hres)
+    out1, cnt1 = st.split_result(hres)
+    assert int(cnt1.item()) == 2
+    got = torch.empty_like(st.out[w.layers - 1])
+    got.copy_(st.out[w.layers - 1])
+    torch.cuda.synchronize()
+    assert ctx.get_device_error() == 0
+    assert torch.equal(out1, got.cpu())
+    out = out1.to(torch.float64).numpy()
+    for b in range(3):
+        ref = hx.oracle_row(w, 1, w.layers - 1, b)
+        want = ref["full"] if b != 1 else ref["local"]
+        hx.assert_close(out[b], want, *hx.tol(w), what=f"run_io row {b}")
+    st.close()
