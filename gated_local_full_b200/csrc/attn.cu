@@ -10,19 +10,28 @@
 //   * The work of one launch is the concatenation of "segments", one per
 //     (row, KV head), each a run of 16-token tiles of [2][16][d] elements
 //     (K rows then V rows, contiguous in both the ring and the paged cache).
-//     The total is split evenly over a persistent grid sized to the SMs, so a
-//     batch-1 128K request and a 32-request mixed batch both fill the GPU.
+//     A persistent grid sized to the SMs takes it: either each segment gets
+//     its own CTAs in proportion to its length (aligned), with the last
+//     tiles of a long segment in a pool that CTAs draw from one at a time,
+//     or the tile space is split evenly (plan.cuh).
 //   * Each warp streams its own tiles through NS shared-memory stages with
 //     cp.async.bulk (TMA bulk copies) completing on mbarriers; waits are
 //     bounded and a timeout is recorded, never trapped.
-//   * q.k: every lane owns d/32 dimensions; the 16*G partial dot products of
-//     a tile are reduced across the warp with a transposing butterfly, leaving
-//     one score per lane. Online softmax in base 2 (q pre-scaled by
-//     log2(e)/sqrt(d)), fp32 accumulation on the CUDA cores: with G = 2 query
-//     heads per KV head the contraction is too thin for tensor cores.
-//   * Warps of a CTA merge their states in shared memory; CTAs sharing a
-//     segment write (m, l, acc) partials and the last one to take the
-//     segment's ticket merges them and writes the output.
+//   * q.k: a K/V row is LPR 16-byte chunks; lane (row group, chunk) holds its
+//     chunk's dimensions of the G query heads in fp32 pairs and multiplies
+//     with packed FMAs; a transposing butterfly over the row group's lanes
+//     leaves one score per lane. Online softmax in base 2 (log2(e)/sqrt(d)
+//     folded into the scores), fp32 accumulation on the CUDA cores: with
+//     G = 2 query heads per KV head the contraction is too thin for tensor
+//     cores.
+//   * Warps of a CTA merge their states in shared memory. Then either CTAs
+//     sharing a segment write (m, l, acc) partials and the last one to take
+//     the segment's ticket merges them and writes the output, or (Local at
+//     small batch) one thread-block cluster serves each segment and its
+//     ranks merge through distributed shared memory.
+//   * Launches chain with programmatic dependent launch; before its
+//     dependency wait a kernel only warms L2 with the K/V it will read.
+
 #include <mutex>
 
 #include <cooperative_groups.h>
@@ -57,8 +66,6 @@ using namespace oda;
 namespace {
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per barrier wait
-
-
 
 struct AttnArgs {
   const void* q;
