@@ -529,7 +529,9 @@ def run_oda(args, rank, ws, local):
     # ---- end to end: host records in, result out, every step
     e2e = None
     if not args.no_e2e:
-        n_e2e = min(K, 256)
+        # the same K steps as the device-timed run (same Full calls), fed from
+        # pinned host memory one step at a time
+        n_e2e = K
         hrec = st.new_records(n_e2e, pin=True)
         hrec.copy_(recs[W:W + n_e2e].cpu())
         res = torch.empty((w.batch, w.hq, w.d), dtype=torch.bfloat16).pin_memory()
