@@ -483,6 +483,7 @@ def run_oda(args, rank, ws, local):
     barrier(ws)
     elapsed = e0.elapsed_time(e1) / 1000.0
     clocks = sampler.summary(h0, h1)
+    sampler.stop()              # nvidia-smi no longer competes with the legs below
     err = ctx.get_device_error()
     t_max = max_over_ranks(elapsed, ws)
     timed = list(range(W, W + K))
@@ -567,7 +568,6 @@ def run_oda(args, rank, ws, local):
                "d2h_bytes_per_step": int(res.numel() * res.element_size() + 4),
                "steps": n_e2e}
 
-    sampler.stop()
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline and not dense:
         steps = cpu_sample_steps(timed, flags, args.cpu_steps)
