@@ -18,7 +18,7 @@ Parity status
   gelu_erf ............................. pinned (erf closed-form values)
   recall_score ......................... parity unpinned: the pages give the
       head's inputs and parameter count but not its architecture; the
-      6144 -> 4096 -> 1 GELU MLP is this build's stated choice. Pinned only
+      6144 -> 4096 -> 1 GELU MLP is this library's stated choice. Pinned only
       through special cases (W1 = 0, a single hidden unit).
 """
 
@@ -132,7 +132,7 @@ def full_attention(q, K, V, t: int, flops: Optional[FlopCounter] = None):
 # ---------------------------------------------------------------------------
 # Recall head R_psi(h_{t-1}, E(x_t), h^L_t) ([SUM] Methodology, recall-score
 # equation; [EXPL] Jargon / Recall head). The pages fix the three inputs and
-# their order, not the architecture. This build's head: concat -> Linear ->
+# their order, not the architecture. This library's head: concat -> Linear ->
 # GELU (erf form) -> Linear to one score.
 # ---------------------------------------------------------------------------
 
