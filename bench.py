@@ -58,10 +58,13 @@ def parse():
                     help="context length t at the first step (the headline is 131072)")
     ap.add_argument("--rate", type=float, default=0.125,
                     help="Full-call rate: Bernoulli per step (the headline is 0.125)")
-    ap.add_argument("--mode", choices=["oda", "full-only"], default="oda",
+    ap.add_argument("--mode", choices=["oda", "full-only", "recall-loss"], default="oda",
                     help="full-only: every step appends and runs Full attention in every "
                          "layer, no Local, recall head or gate (dense decode, for the "
-                         "speedup and the short-context crossover)")
+                         "speedup and the short-context crossover); recall-loss: the recall "
+                         "head's training objective over --positions positions")
+    ap.add_argument("--positions", type=int, default=1 << 24,
+                    help="positions per recall-loss call (--mode recall-loss)")
     return ap.parse_args()
 
 
@@ -405,6 +408,51 @@ def config_block(w, args, ws):
 # our arm
 # ----------------------------------------------------------------------------
 
+def run_recall_loss(args, rank, ws, local):
+    """The recall head's training objective (oda_recall_loss) over
+    --positions seeded synthetic positions: 12 bytes read per position."""
+    import torch
+    from gated_local_full_b200 import oda
+    torch.cuda.set_device(local)
+    n, K, W = args.positions, args.steps, args.warmup
+    gen = torch.Generator(device="cuda").manual_seed(7 + rank)
+    q = torch.randn(n, device="cuda", generator=gen) * 2.0
+    lf = torch.randn(n, device="cuda", generator=gen) * 1.5 - 2.0
+    ll = lf - (torch.randn(n, device="cuda", generator=gen) + 0.1)
+    cfg = oda.make_config(layers=1, max_batch=1, hq=2, hkv=1, head_dim=64, sink=4, window=16,
+                          dtype="f32", max_blocks_per_seq=4, num_blocks=4)
+    ctx = oda.OdaContext(cfg)
+    loss = torch.zeros(1, device="cuda")
+    nf = torch.zeros(1, dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream()
+    for _ in range(W):
+        ctx.recall_loss(q, lf, ll, 0.0, loss, nf)
+    torch.cuda.synchronize()
+    barrier(ws)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(K):
+        ctx.recall_loss(q, lf, ll, 0.0, loss, nf)
+    b.record(stream)
+    torch.cuda.synchronize()
+    t = max_over_ranks(a.elapsed_time(b) / 1000.0, ws)
+    err = ctx.get_device_error()
+    ctx.close()
+    if rank == 0:
+        hbm, kind = peaks()
+        gbs = 12.0 * n * K * ws / t / 1e9
+        print(json.dumps({
+            "metric": "recall-head training objective GB/s (12 B per position)", "value": gbs,
+            "unit": "GB/s", "n_gpus": ws, "steps": K, "warmup": W,
+            "ms_per_step": 1000.0 * t / K, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32 (f64 sum)", "data": "synthetic (seeded)",
+            "config": {"workload": f"oda_recall_loss over {n} positions", "positions": n,
+                       "l2": "inputs of %d MB exceed the 126 MB L2" % (12 * n // 10**6)},
+            "roofline": {"bound": "hbm", "achieved": gbs / ws, "peak": hbm, "unit": "GB/s",
+                         "frac": gbs / ws / hbm, "traffic": None, "peak_kind": kind},
+            "device_error": err}), flush=True)
+
+
 def run_oda(args, rank, ws, local):
     import torch
 
@@ -613,6 +661,8 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, rank, ws)
+        elif args.mode == "recall-loss":
+            run_recall_loss(args, rank, ws, local)
         else:
             run_oda(args, rank, ws, local)
     finally:

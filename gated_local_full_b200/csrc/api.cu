@@ -111,6 +111,13 @@ oda_status oda_create(const oda_config* cfg, oda_ctx** out) {
           cudaSuccess)
     s = ODA_ERR_CUDA;
   if (s == ODA_OK) s = oda_impl::recall_setup(ctx);
+  if (s == ODA_OK) {
+    // recall-loss reduction: block sums (f64), block counts (i32), one ticket
+    const size_t tb = (size_t)oda::kTrainMaxBlocks * (sizeof(double) + sizeof(int)) + 16;
+    if (cudaMalloc(&ctx->train_scratch, tb) != cudaSuccess ||
+        cudaMemset(ctx->train_scratch, 0, tb) != cudaSuccess)
+      s = ODA_ERR_CUDA;
+  }
   if (s == ODA_OK && cudaDeviceSynchronize() != cudaSuccess) s = ODA_ERR_CUDA;
   if (s != ODA_OK) {
     oda_destroy(ctx);
@@ -129,6 +136,7 @@ oda_status oda_destroy(oda_ctx* ctx) {
   cudaFree(ctx->recall_partials);
   cudaFree(ctx->recall_tickets);
   cudaFree(ctx->plan_local);
+  cudaFree(ctx->train_scratch);
   free(ctx);
   return ODA_OK;
 }
@@ -196,6 +204,15 @@ oda_status oda_recall_score(oda_ctx* ctx, const void* h_prev, const void* emb,
   if (H < 1 || hidden < 1) return ODA_ERR_ARG;
   return oda_impl::launch_recall(ctx, h_prev, emb, h_local, H, W1, b1, w2, b2, hidden, scores, B,
                                  static_cast<cudaStream_t>(stream));
+}
+
+oda_status oda_recall_loss(oda_ctx* ctx, const float* q, const float* logp_full,
+                           const float* logp_local, float lambda, int64_t n, float* loss,
+                           int32_t* n_full, oda_stream stream) {
+  if (!ctx || !q || !logp_full || !logp_local || !loss || !n_full || n < 1) return ODA_ERR_ARG;
+  if (n > (int64_t)INT32_MAX) return ODA_ERR_SHAPE;
+  return oda_impl::launch_recall_loss(ctx, q, logp_full, logp_local, lambda, (long long)n, loss,
+                                      n_full, static_cast<cudaStream_t>(stream));
 }
 
 oda_status oda_gate(oda_ctx* ctx, const float* scores, float theta, int B, uint8_t* flags,

@@ -27,6 +27,7 @@ struct oda_ctx {
   float* recall_partials;    // recall-head split partials
   int recall_parts_cap;      // capacity of recall_partials in floats
   int recall_cluster_max;    // largest cluster for the recall head's split-K (0: none)
+  void* train_scratch;       // recall-loss block sums [kTrainMaxBlocks] f64, counts, ticket
   int* plan_local;           // partition shared by a step's Local launches
   int local_cluster_max;     // largest cluster for the cluster-merge Local kernel (0: none)
   int local_wide_cluster_max;  // the same for its one-tile-per-warp shape
@@ -34,6 +35,8 @@ struct oda_ctx {
 };
 
 namespace oda {
+
+constexpr int kTrainMaxBlocks = 1024;   // blocks of the recall-loss reduction
 
 // ----------------------------------------------------------------- host utils
 #define ODA_CUDA_TRY(expr)                                   \
@@ -209,5 +212,8 @@ oda_status launch_recall(oda_ctx* ctx, const void* h_prev, const void* emb, cons
                          int H, const void* W1, const float* b1, const float* w2, float b2,
                          int hidden, float* scores, int B, cudaStream_t st);
 oda_status recall_setup(oda_ctx* ctx);
+oda_status launch_recall_loss(oda_ctx* ctx, const float* q, const float* lpf, const float* lpl,
+                              float lam, long long n, float* loss, int32_t* n_full,
+                              cudaStream_t st);
 oda_status launch_wait_selftest(oda_ctx* ctx, uint64_t timeout_ns, cudaStream_t st);
 }  // namespace oda_impl

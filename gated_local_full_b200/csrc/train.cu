@@ -1,0 +1,120 @@
+// The recall head's training objective on the device.
+//
+// [SUM] Methodology / training the recall head: the access gain of a
+// position is g_t = log p^F_t(x_{t+1}) - log p^L_t(x_{t+1}) (how much Full
+// attention raises the next token's log-probability); the head regresses
+// y_t = T(g_t - lambda) with T(u) = sign(u) log(1 + |u|), under a Huber loss
+// with transition point 1; a step pays for Full exactly when g_t > lambda.
+// For n positions this kernel returns the mean loss and that count.
+//
+// The work is one pass over three float arrays (12 bytes per position), so it
+// is bound by HBM: six CTAs per SM stream them with 16-byte loads, each thread
+// keeps a float64 sum, blocks reduce in a fixed order, and the last block to
+// take the ticket adds the block sums in block order, so the result is the
+// same run to run.
+#include "oda_internal.cuh"
+
+using namespace oda;
+
+namespace {
+
+constexpr int kThreads = 256;
+
+__device__ __forceinline__ float signed_log1p(float u) { return copysignf(log1pf(fabsf(u)), u); }
+
+__device__ __forceinline__ double huber1(float r) {
+  const double a = fabs((double)r);
+  return a <= 1.0 ? 0.5 * a * a : a - 0.5;
+}
+
+// One position: the count of g > lambda and the Huber term.
+__device__ __forceinline__ void position(float qv, float f, float l, float lam, double& s, int& c) {
+  const float g = f - l;                             // access gain, fp32
+  c += g > lam ? 1 : 0;                              // Full pays off (strict)
+  s += huber1(qv - signed_log1p(g - lam));
+}
+
+__global__ void __launch_bounds__(kThreads)
+recall_loss_kernel(const float* __restrict__ q, const float* __restrict__ lpf,
+                   const float* __restrict__ lpl, float lam, long long n, int vec,
+                   double* __restrict__ bsum, int* __restrict__ bcnt, int* __restrict__ ticket,
+                   float* __restrict__ loss, int32_t* __restrict__ n_full) {
+  __shared__ double ssum[kThreads / 32];
+  __shared__ int scnt[kThreads / 32];
+  __shared__ int last;
+  pdl_wait();
+  pdl_launch_dependents();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const long long stride = (long long)gridDim.x * kThreads;
+  const long long first = blockIdx.x * (long long)kThreads + tid;
+  double s = 0.0;
+  int c = 0;
+  // 16-byte loads of four positions of each array, streamed past L1/L2
+  const long long n4 = vec ? n / 4 : 0;
+  const float4* q4 = reinterpret_cast<const float4*>(q);
+  const float4* f4 = reinterpret_cast<const float4*>(lpf);
+  const float4* l4 = reinterpret_cast<const float4*>(lpl);
+#pragma unroll 2
+  for (long long i = first; i < n4; i += stride) {
+    const float4 a = __ldcs(q4 + i), f = __ldcs(f4 + i), l = __ldcs(l4 + i);
+    position(a.x, f.x, l.x, lam, s, c);
+    position(a.y, f.y, l.y, lam, s, c);
+    position(a.z, f.z, l.z, lam, s, c);
+    position(a.w, f.w, l.w, lam, s, c);
+  }
+  for (long long i = n4 * 4 + first; i < n; i += stride) position(q[i], lpf[i], lpl[i], lam, s, c);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    s += __shfl_xor_sync(0xffffffffu, s, o);
+    c += __shfl_xor_sync(0xffffffffu, c, o);
+  }
+  if (lane == 0) { ssum[warp] = s; scnt[warp] = c; }
+  __syncthreads();
+  if (tid == 0) {
+    double t = 0.0;
+    int k = 0;
+    for (int w = 0; w < kThreads / 32; ++w) { t += ssum[w]; k += scnt[w]; }
+    bsum[blockIdx.x] = t;
+    bcnt[blockIdx.x] = k;
+    __threadfence();
+    last = atomicAdd(ticket, 1) == (int)gridDim.x - 1;
+  }
+  __syncthreads();
+  if (last && tid == 0) {
+    __threadfence();
+    double t = 0.0;
+    long long k = 0;
+    for (int b = 0; b < (int)gridDim.x; ++b) {
+      t += __ldcg(bsum + b);
+      k += __ldcg(bcnt + b);
+    }
+    *loss = (float)(t / (double)n);
+    *n_full = (int32_t)k;
+    *ticket = 0;
+  }
+}
+
+}  // namespace
+
+namespace oda_impl {
+
+oda_status launch_recall_loss(oda_ctx* ctx, const float* q, const float* lpf, const float* lpl,
+                              float lam, long long n, float* loss, int32_t* n_full,
+                              cudaStream_t st) {
+  long long grid = (n + kThreads * 8 - 1) / (kThreads * 8);   // >= 8 positions per thread
+  const long long cap = (long long)ctx->num_sms * 6;
+  if (grid > cap) grid = cap;
+  if (grid < 1) grid = 1;
+  double* bsum = reinterpret_cast<double*>(ctx->train_scratch);
+  int* bcnt = reinterpret_cast<int*>(bsum + kTrainMaxBlocks);
+  int* ticket = bcnt + kTrainMaxBlocks;
+  if (grid > kTrainMaxBlocks) grid = kTrainMaxBlocks;
+  const int vec = ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(lpf) |
+                    reinterpret_cast<uintptr_t>(lpl)) & 15u) == 0;
+  return launch_pdl(recall_loss_kernel, dim3((unsigned)grid), dim3(kThreads), 0, st, q, lpf, lpl,
+                    lam, n, vec, bsum, bcnt, ticket, loss, n_full) == cudaSuccess
+             ? ODA_OK
+             : ODA_ERR_CUDA;
+}
+
+}  // namespace oda_impl

@@ -28,7 +28,7 @@ STATUS_NAMES = {0: "ODA_OK", 1: "ODA_ERR_ARG", 2: "ODA_ERR_SHAPE", 3: "ODA_ERR_D
 # Every symbol include/oda.h declares.
 EXPORTS = (
     "oda_layout", "oda_create", "oda_destroy", "oda_append_kv", "oda_ring_init",
-    "oda_local_attn", "oda_recall_score", "oda_gate", "oda_full_attn_gated",
+    "oda_local_attn", "oda_recall_score", "oda_recall_loss", "oda_gate", "oda_full_attn_gated",
     "oda_get_device_error", "oda_selftest_wait_timeout", "oda_step_run",
     "oda_step_graph_create", "oda_step_graph_launch", "oda_step_graph_run_io",
     "oda_step_graph_destroy", "oda_version",
@@ -87,6 +87,7 @@ def lib() -> ctypes.CDLL:
         "oda_local_attn": [vp, c_int, vp, vp, vp, vp, vp, c_int, vp],
         "oda_recall_score": [vp, vp, vp, vp, c_int, vp, vp, vp, c_float, c_int, vp, c_int, vp],
         "oda_gate": [vp, vp, c_float, c_int, vp, vp, vp, vp],
+        "oda_recall_loss": [vp, vp, vp, vp, c_float, c_int64, vp, vp, vp],
         "oda_full_attn_gated": [vp, c_int, vp, vp, vp, vp, vp, vp, vp, vp, c_int, vp],
         "oda_get_device_error": [vp, vp, POINTER(c_int)],
         "oda_selftest_wait_timeout": [vp, c_uint64, vp],
@@ -235,6 +236,15 @@ class OdaContext:
         _check(lib().oda_recall_score(self.handle, ptr(h_prev), ptr(emb), ptr(h_local), H,
                                       ptr(W1), ptr(b1), ptr(w2), float(b2), hidden, ptr(scores),
                                       B, _stream(stream)), "oda_recall_score")
+
+    def recall_loss(self, q, logp_full, logp_local, lam, loss, n_full, stream=None):
+        """Mean Huber_1(q - T(g - lam)) and #{g > lam}, g = logp_full - logp_local."""
+        n = q.numel()
+        if logp_full.numel() != n or logp_local.numel() != n:
+            raise ValueError("recall_loss: q, logp_full and logp_local differ in length")
+        _check(lib().oda_recall_loss(self.handle, ptr(q), ptr(logp_full), ptr(logp_local),
+                                     float(lam), n, ptr(loss), ptr(n_full), _stream(stream)),
+               "oda_recall_loss")
 
     def gate(self, scores, theta, B, flags, idx, count, stream=None):
         _check(lib().oda_gate(self.handle, ptr(scores), float(theta), B, ptr(flags), ptr(idx),

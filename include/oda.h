@@ -186,6 +186,24 @@ oda_status oda_recall_score(oda_ctx* ctx, const void* h_prev, const void* emb,
                             float* scores, int B, oda_stream stream);
 
 /*
+ * Training objective of the recall head ([SUM] Methodology, training the
+ * recall head; an offline step, not part of a decode step). For n positions:
+ *   g_t = logp_full[t] - logp_local[t]          access gain (float32),
+ *   y_t = T(g_t - lambda),  T(u) = sign(u) log(1 + |u|),
+ *   *loss   = (1/n) sum_t Huber_1(q[t] - y_t)   (Huber with transition 1),
+ *   *n_full = #{t : g_t > lambda}               (steps where Full pays off).
+ *   q, logp_full, logp_local  device float [n] (recall scores; next-token
+ *                             log-probabilities under Full and under Local)
+ *   loss     device float [1];  n_full  device int32 [1]
+ * The sum is kept in float64 and reduced in a fixed order (deterministic).
+ * 1 <= n <= 2^31 - 1, else ODA_ERR_ARG / ODA_ERR_SHAPE. Uses the context's
+ * scratch: calls on one context must not overlap.
+ */
+oda_status oda_recall_loss(oda_ctx* ctx, const float* q, const float* logp_full,
+                           const float* logp_local, float lambda, int64_t n, float* loss,
+                           int32_t* n_full, oda_stream stream);
+
+/*
  * Threshold gate ([SUM] Methodology: recompute with Full iff q_t > theta;
  * default theta = 0) with device-side compaction ([SUM] Efficient Execution:
  * GPU-side conditional execution, no host round trip):
