@@ -500,7 +500,7 @@ def run_oda(args, rank, ws, local):
                           dw.ring, w.batch)
             for l in range(w.layers):
                 ctx.full_attn_gated(l, st.q[l], st.seq_lens, dw.block_table, dw.cache, idx_all,
-                                    cnt_all, st.out[l], None, w.batch)
+                                    cnt_all, st.out[l], None, w.batch, inputs_ready=l > 0)
 
         side = torch.cuda.Stream()
         side.wait_stream(stream)
@@ -562,14 +562,14 @@ def run_oda(args, rank, ws, local):
             sl = st.record_view(recs, i, "seq_lens")
             for l in range(w.layers):
                 ctx.full_attn_gated(l, q[l], sl, dw.block_table, dw.cache, idx0, cnt1, outb,
-                                    None, w.batch)
+                                    None, w.batch, inputs_ready=l > 0)
 
     def run_local():
         for i in timed[:16]:
             q = st.record_view(recs, i, "q")
             sl = st.record_view(recs, i, "seq_lens")
             for l in range(w.layers):
-                ctx.local_attn(l, q[l], sl, dw.ring, outb, None, w.batch)
+                ctx.local_attn(l, q[l], sl, dw.ring, outb, None, w.batch, inputs_ready=l > 0)
 
     full_s, n_full = replay_seconds(torch, run_full, stream), len(fl_steps) * w.layers
     local_s, n_local = replay_seconds(torch, run_local, stream), min(K, 16) * w.layers

@@ -2,6 +2,9 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <mutex>
+#include <vector>
+
 #include "oda_internal.cuh"
 #include "plan.cuh"
 
@@ -48,6 +51,63 @@ __global__ void wait_selftest_kernel(uint64_t timeout_ns, int* err) {
 }
 
 }  // namespace
+
+namespace oda {
+
+namespace attr_cache {
+struct SmemLimit {
+  int dev;
+  const void* fn;
+  size_t bytes;
+};
+struct OccEntry {
+  int dev;
+  const void* fn;
+  int threads;
+  size_t smem;
+  int occ;
+};
+std::mutex g_attr_mu;
+std::vector<SmemLimit> g_smem_limits;
+std::vector<OccEntry> g_occ;
+}  // namespace attr_cache
+using namespace attr_cache;
+
+cudaError_t raise_smem_limit(const void* fn, size_t bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(g_attr_mu);
+  for (SmemLimit& l : g_smem_limits) {
+    if (l.dev == dev && l.fn == fn) {
+      if (l.bytes >= bytes) return cudaSuccess;
+      e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+      if (e == cudaSuccess) l.bytes = bytes;
+      return e;
+    }
+  }
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) g_smem_limits.push_back(SmemLimit{dev, fn, bytes});
+  return e;
+}
+
+cudaError_t occupancy_cached(int* occ, const void* fn, int threads, size_t smem) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(g_attr_mu);
+  for (const OccEntry& o : g_occ) {
+    if (o.dev == dev && o.fn == fn && o.threads == threads && o.smem == smem) {
+      *occ = o.occ;
+      return cudaSuccess;
+    }
+  }
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(occ, fn, threads, smem);
+  if (e == cudaSuccess) g_occ.push_back(OccEntry{dev, fn, threads, smem, *occ});
+  return e;
+}
+
+}  // namespace oda
 
 namespace oda_impl {
 oda_status launch_wait_selftest(oda_ctx* ctx, uint64_t timeout_ns, cudaStream_t st) {
@@ -168,29 +228,34 @@ oda_status oda_ring_init(oda_ctx* ctx, int layer_begin, int layer_end, const int
 }
 
 oda_status oda_local_attn(oda_ctx* ctx, int layer, const void* q, const int32_t* seq_lens,
-                          const void* ring, void* out, float* lse, int B, oda_stream stream) {
+                          const void* ring, void* out, float* lse, int B, unsigned flags,
+                          oda_stream stream) {
   if (!ctx) return ODA_ERR_ARG;
   oda_status s = check_batch(ctx, B);
   if (s != ODA_OK) return s;
   if (layer < 0 || layer >= ctx->cfg.layers) return ODA_ERR_ARG;
+  if (flags & ~ODA_ATTN_INPUTS_READY) return ODA_ERR_ARG;
   if (B == 0) return ODA_OK;
   if (!q || !seq_lens || !ring || !out) return ODA_ERR_ARG;
   return oda_impl::launch_attn(ctx, true, layer, q, seq_lens, ring, nullptr, nullptr, nullptr, out,
-                               lse, B, static_cast<cudaStream_t>(stream));
+                               lse, B, static_cast<cudaStream_t>(stream), nullptr,
+                               (flags & ODA_ATTN_INPUTS_READY) != 0);
 }
 
 oda_status oda_full_attn_gated(oda_ctx* ctx, int layer, const void* q, const int32_t* seq_lens,
                                const int32_t* block_table, const void* kv_cache,
                                const int32_t* idx, const int32_t* count, void* out, float* lse,
-                               int B, oda_stream stream) {
+                               int B, unsigned flags, oda_stream stream) {
   if (!ctx) return ODA_ERR_ARG;
   oda_status s = check_batch(ctx, B);
   if (s != ODA_OK) return s;
   if (layer < 0 || layer >= ctx->cfg.layers) return ODA_ERR_ARG;
+  if (flags & ~ODA_ATTN_INPUTS_READY) return ODA_ERR_ARG;
   if (B == 0) return ODA_OK;
   if (!q || !seq_lens || !block_table || !kv_cache || !idx || !count || !out) return ODA_ERR_ARG;
   return oda_impl::launch_attn(ctx, false, layer, q, seq_lens, kv_cache, block_table, idx, count,
-                               out, lse, B, static_cast<cudaStream_t>(stream));
+                               out, lse, B, static_cast<cudaStream_t>(stream), nullptr,
+                               (flags & ODA_ATTN_INPUTS_READY) != 0);
 }
 
 oda_status oda_recall_score(oda_ctx* ctx, const void* h_prev, const void* emb,

@@ -92,6 +92,7 @@ struct AttnArgs {
   int* dyn;                     // per segment: tiles handed out dynamically (reset by the last)
   const int* plan;              // precomputed partition, or null: compute it here
   int cluster;                  // cluster mode: CTAs per segment (= cluster size)
+  int early;                    // stage the first tiles before the dependency wait
   int* err;
 };
 
@@ -101,23 +102,34 @@ struct Chunk;
 
 template <>
 struct Chunk<__nv_bfloat16> {
-  static __device__ __forceinline__ void load(const __nv_bfloat16* p, float2 (&x)[4]) {
-    const uint4 w = *reinterpret_cast<const uint4*>(p);
+  static __device__ __forceinline__ void widen(const uint4 w, float2 (&x)[4]) {
     bf16x2_to_f32(w.x, x[0].x, x[0].y);
     bf16x2_to_f32(w.y, x[1].x, x[1].y);
     bf16x2_to_f32(w.z, x[2].x, x[2].y);
     bf16x2_to_f32(w.w, x[3].x, x[3].y);
   }
+  static __device__ __forceinline__ void load(const __nv_bfloat16* p, float2 (&x)[4]) {
+    widen(*reinterpret_cast<const uint4*>(p), x);
+  }
 };
 
 template <>
 struct Chunk<float> {
+  static __device__ __forceinline__ void widen(const uint4 w, float2 (&x)[2]) {
+    x[0] = make_float2(__uint_as_float(w.x), __uint_as_float(w.y));
+    x[1] = make_float2(__uint_as_float(w.z), __uint_as_float(w.w));
+  }
   static __device__ __forceinline__ void load(const float* p, float2 (&x)[2]) {
-    const float4 w = *reinterpret_cast<const float4*>(p);
-    x[0] = make_float2(w.x, w.y);
-    x[1] = make_float2(w.z, w.w);
+    widen(*reinterpret_cast<const uint4*>(p), x);
   }
 };
+
+// A query chunk from global memory (L2, issued at once: see ld_cg_v4), widened
+// where it is first needed.
+template <typename T>
+__device__ __forceinline__ uint4 q_chunk(const T* p) {
+  return ld_cg_v4(p);
+}
 
 // Bits [lo, hi) of a 16-bit tile mask whose bit 0 is slot `base`.
 __device__ __forceinline__ uint32_t range_bits(int lo, int hi, int base) {
@@ -214,6 +226,9 @@ attn_kernel(const AttnArgs a) {
   float* racc = reinterpret_cast<float*>(
       (reinterpret_cast<uintptr_t>(badst + W * NS) + 15) & ~uintptr_t(15));  // CL: [cs][G*D/cs]
   float* rml = racc + G * D;                   // CL: [16][G] pushed (m, l) pairs
+  constexpr int QCH = G * D * (int)sizeof(T) / 16;  // 16-byte chunks of one segment's queries
+  uint4* sq = reinterpret_cast<uint4*>(rml + 32 * G);   // [QCH] the current segment's queries
+  int* st_t = reinterpret_cast<int*>(sq + QCH);         // cluster mode: the row's t
 
   const int tid = threadIdx.x;
   const int lane = tid & 31;
@@ -223,18 +238,35 @@ attn_kernel(const AttnArgs a) {
   const int hq = a.hkv * G;
   if (tid < W * NS) mbar_init(smem_addr(&bars[tid]), 1);
   fence_mbar_init();
+  // Early mode: the caller guarantees that the K/V source, the lengths, the
+  // block table and the compacted ids were complete before the previous
+  // kernel on the stream passed its own dependency wait (every kernel of this
+  // library waits before it lets dependents start), so this launch works out
+  // its partition and issues its first tile copies into shared memory before
+  // its own wait. The queries, the scratch (partials, tickets, pool counters)
+  // and the outputs are touched only after the wait.
+  const bool early = a.early != 0;
   if constexpr (CL) {
     cluster_arrive_relaxed();                    // "started": waited for before any remote store
-    // Before the dependency wait, warm L2 with this rank's share of a full
-    // ring (its share once t >= w). This reads no value: L2 is the point of
-    // coherence, so the loads after the wait still see every earlier write,
-    // and the prefetch overlaps the tail of the preceding kernel.
     const int cs = a.cluster;
     const int sg = (int)blockIdx.x / cs, rank = (int)blockIdx.x % cs;
-    const int rb = a.ring_blocks;
-    const int k0 = (rank * rb) / cs, k1 = ((rank + 1) * rb) / cs;
-    const T* base = reinterpret_cast<const T*>(a.kv) + (long long)sg * rb * TILE_ELEMS;
-    for (int k = k0 + tid; k < k1; k += W * 32) bulk_prefetch_l2(base + (long long)k * TILE_ELEMS, TILE_BYTES);
+    if (early) {
+      // this segment's queries into L2 (a prefetch returns no value)
+      if (tid == 0)
+        bulk_prefetch_l2(reinterpret_cast<const T*>(a.q) +
+                             ((long long)(sg / a.hkv) * hq + (sg % a.hkv) * G) * D,
+                         G * D * (int)sizeof(T));
+    } else {
+      // Before the dependency wait, warm L2 with this rank's share of a full
+      // ring (its share once t >= w). This reads no value: L2 is the point of
+      // coherence, so the loads after the wait still see every earlier write,
+      // and the prefetch overlaps the tail of the preceding kernel.
+      const int rb = a.ring_blocks;
+      const int k0 = (rank * rb) / cs, k1 = ((rank + 1) * rb) / cs;
+      const T* base = reinterpret_cast<const T*>(a.kv) + (long long)sg * rb * TILE_ELEMS;
+      for (int k = k0 + tid; k < k1; k += W * 32)
+        bulk_prefetch_l2(base + (long long)k * TILE_ELEMS, TILE_BYTES);
+    }
   }
   // ------------------------------------------------------- rows, partition
   // Either read the plan another kernel wrote once for every launch that
@@ -284,13 +316,13 @@ attn_kernel(const AttnArgs a) {
 #if ODA_PREFETCH_TILES > 0
   static_assert(ODA_PREFETCH_TILES <= 32, "one prefetched tile per lane of warp 0");
   if constexpr (!CL) {
-    // Before the dependency wait, warp 0 works out the partition from values
+    // Without early staging: before the dependency wait, warp 0 works out the partition from values
     // that the preceding launch may still be writing, and warms L2 with the
     // first tiles of this CTA's static share. Nothing read here is used after
     // the wait (the partition is worked out again), and an L2 prefetch reads
     // no value, so a stale guess only costs bandwidth; every address is
     // bounds-checked like the loads proper.
-    if (warp == 0) {
+    if (!early && warp == 0) {
       partition(false);
       __syncwarp();
       const int nr = sinfo[0], tot = sinfo[1];
@@ -327,8 +359,10 @@ attn_kernel(const AttnArgs a) {
     }
   }
 #endif
-  pdl_wait();
-  pdl_launch_dependents();
+  if (!early) {
+    pdl_wait();
+    pdl_launch_dependents();
+  }
   float* pacc = a.partials;                                         // [max_parts][G][D]
   float* pml = a.partials + (size_t)a.max_parts * G * D;            // [max_parts][G][2]
 
@@ -398,12 +432,7 @@ attn_kernel(const AttnArgs a) {
       }
     }
   };
-  // (cluster mode never leaves early: every CTA takes part in the merge)
   const bool has_work = nrows > 0 && total > 0 && lo < hi;
-  if (!CL && !has_work) return;
-  if (CL && !has_work) {
-    cluster_push(false);                         // an empty state: m = -inf, l = acc = 0
-  } else {
 
   // K/V is read once per launch: stream it through L2 (the ring too, so no
   // layer's window stays resident from one step to the next)
@@ -416,41 +445,17 @@ attn_kernel(const AttnArgs a) {
   // pool: a warp that finishes its static share takes pool tiles one at a
   // time from the segment's counter (two grabs kept in flight), so warps
   // that stream faster take more and the segment's CTAs finish together.
+  // The pool counters are scratch: they are touched only after the wait.
   Cursor prod;
-  prod.k = lo;
-  locate(rowstart, nrows, a.hkv, lo, prod);
-  const int seg_b = rowb[prod.i];
-  const int seg_nt = prod.nt;
-  const int seg_s0 = prod.s1 - prod.nt;
-  const int sigma0 = prod.i * a.hkv + prod.g;
-  int pool0 = seg_nt;                        // first pool tile (relative); == nt: no pool
-  if (!CL && aligned && seg_nt >= 8 * nparts_al * W) {
-    pool0 = seg_nt - pool_tiles(seg_nt, nparts_al, W);
-    // static share of this CTA within [0, pool0)
-    lo = seg_s0 + (int)(((long long)part_al * pool0) / nparts_al);
-    hi = seg_s0 + (int)(((long long)(part_al + 1) * pool0) / nparts_al);
-  }
-  const bool use_pool = pool0 < seg_nt;
-  // cluster mode has one segment per CTA: its queries and t are loaded
-  // before the first copies are issued, so they land while the copies fly
-  float2 qpre[G][DP2];
-  int tpre = 0;
-  if constexpr (CL) {
-    tpre = a.seq_lens[seg_b];
-#pragma unroll
-    for (int h = 0; h < G; ++h)
-      Chunk<T>::load(reinterpret_cast<const T*>(a.q) +
-                         ((long long)seg_b * hq + prod.g * G + h) * D + li * DPL,
-                     qpre[h]);
-  }
-  int q0 = seg_nt, q1 = seg_nt, qb0 = -1, qb1 = -1;   // lane 0: grabbed pool tiles, blocks
-  auto grab = [&](int& q, int& qb) {                  // lane 0 only
+  prod.k = prod.i = prod.g = prod.nt = prod.s1 = 0;
+  int seg_b = 0, seg_g0 = 0, seg_nt = 0, seg_s0 = 0, sigma0 = 0;
+  int pool0 = 0;                             // first pool tile (relative); == nt: no pool
+  bool use_pool = false;
+  int q0 = 0, q1 = 0, qb0 = -1, qb1 = -1;    // lane 0: grabbed pool tiles, blocks
+  auto grab = [&](int& q, int& qb) {         // lane 0 only, after the dependency wait
     q = pool0 + atomicAdd(&a.dyn[sigma0], 1);
     qb = (!RING && q < seg_nt) ? a.block_table[(long long)seg_b * a.max_blocks + q] : -1;
   };
-  prod.k = lo + warp;
-  if (prod.k >= hi) prod.k = hi;
-  normalize(rowstart, a.hkv, hi, warp, prod);
 
   // Block ids of the producer's next 32 tiles of the current row, one per
   // lane, so the per-tile issue does not wait on a global load.
@@ -517,12 +522,68 @@ attn_kernel(const AttnArgs a) {
 
   int issued = 0;
   bool prod_done = false;
+  if (has_work) {
+    prod.k = lo;
+    locate(rowstart, nrows, a.hkv, lo, prod);
+    seg_b = rowb[prod.i];
+    seg_g0 = prod.g;
+    seg_nt = prod.nt;
+    seg_s0 = prod.s1 - prod.nt;
+    sigma0 = prod.i * a.hkv + prod.g;
+    pool0 = seg_nt;
+    if (!CL && aligned && seg_nt >= 8 * nparts_al * W) {
+      pool0 = seg_nt - pool_tiles(seg_nt, nparts_al, W);
+      // static share of this CTA within [0, pool0)
+      lo = seg_s0 + (int)(((long long)part_al * pool0) / nparts_al);
+      hi = seg_s0 + (int)(((long long)(part_al + 1) * pool0) / nparts_al);
+    }
+    use_pool = pool0 < seg_nt;
+    q0 = q1 = seg_nt;
+    if (!CL && early && tid == 0)
+      // the first segment's queries into L2 (a prefetch returns no value)
+      bulk_prefetch_l2(reinterpret_cast<const T*>(a.q) +
+                           ((long long)seg_b * hq + prod.g * G) * D,
+                       G * D * (int)sizeof(T));
+    prod.k = lo + warp;
+    if (prod.k >= hi) prod.k = hi;
+    normalize(rowstart, a.hkv, hi, warp, prod);
 #pragma unroll 1
-  for (int st2 = 0; st2 < NS; ++st2) {
-    int k, i, g, nt, blk;
-    if (!next_tile(k, i, g, nt, blk)) { prod_done = true; break; }
-    issue(k, i, g, nt, blk, st2);
-    ++issued;
+    for (int st2 = 0; st2 < NS; ++st2) {
+      int k, i, g, nt, blk;
+      if (!next_tile(k, i, g, nt, blk)) { prod_done = true; break; }
+      issue(k, i, g, nt, blk, st2);
+      ++issued;
+    }
+  }
+  if (early) {
+    pdl_wait();
+    pdl_launch_dependents();
+  }
+
+  // (cluster mode never leaves early: every CTA takes part in the merge)
+  if (!CL && !has_work) return;
+  if (CL && !has_work) {
+    cluster_push(false);                         // an empty state: m = -inf, l = acc = 0
+  } else {
+
+  // A segment's queries (and, in cluster mode, its row's t) are read once per
+  // CTA by warp 0 into shared memory: one request per CTA instead of one per
+  // warp keeps the hot lines of q from queueing at their L2 slice. Cluster
+  // mode has one segment per CTA, loaded here while the first copies fly.
+  auto load_q = [&](int row, int g, bool with_t) {   // warp 0; the caller syncs
+    const unsigned char* src = reinterpret_cast<const unsigned char*>(a.q) +
+                               ((long long)row * hq + g * G) * D * (long long)sizeof(T);
+    for (int c = lane; c < QCH; c += 32) sq[c] = q_chunk(reinterpret_cast<const T*>(src + 16 * c));
+    if (with_t && lane == 0) st_t[0] = ld_cg_s32(a.seq_lens + row);
+  };
+  uint4 qraw[G];
+  int tpre = 0;
+  if constexpr (CL) {
+    if (warp == 0) load_q(seg_b, seg_g0, true);
+    __syncthreads();
+#pragma unroll
+    for (int h = 0; h < G; ++h) qraw[h] = sq[h * LPR + li];
+    tpre = st_t[0];
   }
   if (use_pool && lane == 0) {       // after the first copies are in flight
     grab(q0, qb0);
@@ -541,7 +602,7 @@ attn_kernel(const AttnArgs a) {
     const int b = rowb[seg.i];
     int t;
     if (CL) {
-      t = tpre;                                  // loaded before the first copies
+      t = tpre;                                  // loaded once per CTA
       if (t < 1) {
         if (tid == 0 && (int)blockIdx.x % a.cluster == 0) record_error(a.err, ODA_ERR_BOUNDS);
         t = 0;                                   // every slot masked: an empty state
@@ -553,17 +614,14 @@ attn_kernel(const AttnArgs a) {
 
     // this lane's DPL dims of the G query heads (exact, unscaled)
     float2 q2[G][DP2];
+    if constexpr (!CL) {
+      if (warp == 0) load_q(b, seg.g, false);
+      __syncthreads();
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      if constexpr (CL) {
-#pragma unroll
-        for (int e = 0; e < DP2; ++e) q2[h][e] = qpre[h][e];
-      } else {
-        const T* qp = reinterpret_cast<const T*>(a.q) +
-                      ((long long)b * hq + seg.g * G + h) * D + li * DPL;
-        Chunk<T>::load(qp, q2[h]);
-      }
+      for (int h = 0; h < G; ++h) qraw[h] = sq[h * LPR + li];
     }
+#pragma unroll
+    for (int h = 0; h < G; ++h) Chunk<T>::widen(qraw[h], q2[h]);
     float m_run[G], l_run[G];
     float2 acc[G][DP2];
 #pragma unroll
@@ -1072,6 +1130,7 @@ size_t smem_bytes_wn(int max_batch) {
   s += (size_t)W * NS * 4;
   s += (size_t)W * NS;
   s += 16 + (size_t)(G * D + 32 * G) * 4;     // cluster mode: pushed accumulators, (m, l)
+  s += (size_t)G * D * sizeof(T) + 16;          // the segment's queries, t
   return (s + 127) & ~(size_t)127;
 }
 
@@ -1095,10 +1154,9 @@ int cluster_setup(oda_ctx* ctx, int& ctas) {
   const size_t sm = smem_bytes_wn<T, D, G, W, NS>(ctx->cfg.max_batch);
   ctas = 0;
   int occ = 0;
-  if (cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) !=
-          cudaSuccess ||
+  if (raise_smem_limit(reinterpret_cast<const void*>(kc), sm) != cudaSuccess ||
       cudaFuncSetAttribute(kc, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kc, W * 32, sm) != cudaSuccess ||
+      occupancy_cached(&occ, reinterpret_cast<const void*>(kc), W * 32, sm) != cudaSuccess ||
       occ < 1) {
     cudaGetLastError();
     return 0;
@@ -1131,9 +1189,9 @@ template <typename T, int D, int G, bool RING>
 oda_status setup_one(oda_ctx* ctx, int& ctas) {
   auto k = kernel_ptr<T, D, G, RING>();
   const size_t sm = smem_bytes<T, D, G, RING>(ctx->cfg.max_batch);
-  ODA_CUDA_TRY(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
+  ODA_CUDA_TRY(raise_smem_limit(reinterpret_cast<const void*>(k), sm));
   int occ = 0;
-  ODA_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, Shape<T, D, G>::W * 32, sm));
+  ODA_CUDA_TRY(occupancy_cached(&occ, reinterpret_cast<const void*>(k), Shape<T, D, G>::W * 32, sm));
   if (occ < 1) return ODA_ERR_SHAPE;
   ctas = ctx->num_sms * occ;
   if (RING) {
@@ -1255,7 +1313,7 @@ oda_status attn_setup(oda_ctx* ctx) {
 oda_status launch_attn(oda_ctx* ctx, bool ring_mode, int layer, const void* q,
                        const int32_t* seq_lens, const void* kv, const int32_t* block_table,
                        const int32_t* idx, const int32_t* count, void* out, float* lse, int B,
-                       cudaStream_t st, const int* plan) {
+                       cudaStream_t st, const int* plan, bool early) {
   const oda_config& c = ctx->cfg;
   AttnArgs a;
   a.q = q;
@@ -1283,6 +1341,7 @@ oda_status launch_attn(oda_ctx* ctx, bool ring_mode, int layer, const void* q,
   a.dyn = ctx->tickets + (size_t)c.max_batch * c.hkv;
   a.plan = plan;
   a.cluster = 0;
+  a.early = early ? 1 : 0;
   a.err = ctx->err;
   if (ring_mode) return dispatch<true>(c, Launch{ctx, &a, st, true});
   return dispatch<false>(c, Launch{ctx, &a, st, false});
@@ -1372,11 +1431,12 @@ struct LaunchStatic {
   oda_status operator()() {
     auto k = kernel_ptr<T, D, G, RING>();
     const size_t sm = smem_bytes<T, D, G, RING>(max_batch);
-    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) !=
-        cudaSuccess)
+    // the limit only ever rises (a context sized for more rows keeps working),
+    // and the occupancy is asked of the runtime once per size
+    if (raise_smem_limit(reinterpret_cast<const void*>(k), sm) != cudaSuccess)
       return ODA_ERR_CUDA;
     int occ = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, Shape<T, D, G>::W * 32, sm) !=
+    if (occupancy_cached(&occ, reinterpret_cast<const void*>(k), Shape<T, D, G>::W * 32, sm) !=
             cudaSuccess ||
         occ < 1)
       return ODA_ERR_CUDA;
@@ -1447,6 +1507,7 @@ extern "C" oda_status oda_full_attn_gated_static(const oda_config* cfg, int laye
   a.dyn = sd->tickets + kStaticMaxSegments;
   a.plan = nullptr;
   a.cluster = 0;
+  a.early = 0;
   a.err = err ? err : sd->err;
   return dispatch<false>(*cfg, LaunchStatic{&a, sd->num_sms, cfg->max_batch, B, st});
 }

@@ -47,6 +47,16 @@ constexpr int kTrainMaxBlocks = 1024;   // blocks of the recall-loss reduction
 
 inline int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+// A kernel's dynamic shared-memory limit is one value per (function, device)
+// for the whole process, shared by every context and by the allocation-free
+// entry point. raise_smem_limit sets it to at least `bytes` on the current
+// device and never lowers it, so one caller sized for a small batch cannot
+// break another's launches. occupancy_cached returns the resident blocks per
+// SM of `fn` at `threads` threads and `smem` bytes, asked of the runtime once
+// per (device, function, threads, smem). Both are thread safe.
+cudaError_t raise_smem_limit(const void* fn, size_t bytes);
+cudaError_t occupancy_cached(int* occ, const void* fn, int threads, size_t smem);
+
 // ------------------------------------------------------------ device helpers
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
@@ -155,6 +165,23 @@ __device__ __forceinline__ float fast_log2(float x) {
   return y;
 }
 
+// 16-byte global load through L2 only (bypassing L1), issued where it stands:
+// the asm is volatile, so the compiler neither drops nor sinks it below later
+// volatile operations (a load whose result is needed late still leaves early).
+__device__ __forceinline__ uint4 ld_cg_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ int ld_cg_s32(const int* p) {
+  int v;
+  asm volatile("ld.global.cg.s32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
+
 // bf16 pair (packed in a 32-bit word, low half first) -> two floats, exactly.
 __device__ __forceinline__ void bf16x2_to_f32(uint32_t w, float& lo, float& hi) {
   lo = __uint_as_float(w << 16);
@@ -202,7 +229,7 @@ oda_status launch_ring_init(oda_ctx* ctx, int lb, int le, const int32_t* seq_len
 oda_status launch_attn(oda_ctx* ctx, bool ring_mode, int layer, const void* q,
                        const int32_t* seq_lens, const void* kv, const int32_t* block_table,
                        const int32_t* idx, const int32_t* count, void* out, float* lse, int B,
-                       cudaStream_t st, const int* plan = nullptr);
+                       cudaStream_t st, const int* plan = nullptr, bool early = false);
 int attn_min_tiles(oda_ctx* ctx, bool ring_mode);
 oda_status attn_setup(oda_ctx* ctx);
 oda_status launch_gate(oda_ctx* ctx, const float* scores, float theta, int B, uint8_t* flags,

@@ -685,8 +685,7 @@ oda_status recall_setup(oda_ctx* ctx) {
   const size_t max_smem = smem_for(MAX_N, stages_for(MAX_N));
   size_t best = max_smem;
   for (int n = 16; n <= MAX_N; n += 16) best = best > smem_for(n, stages_for(n)) ? best : smem_for(n, stages_for(n));
-  ODA_CUDA_TRY(cudaFuncSetAttribute(recall_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)best));
+  ODA_CUDA_TRY(raise_smem_limit(reinterpret_cast<const void*>(recall_kernel), best));
   const size_t pfl = (size_t)(ctx->num_sms + MAX_MT) * MAX_N * BM + (size_t)MAX_MT * MAX_N;
   ODA_CUDA_TRY(cudaMalloc(&ctx->recall_partials, pfl * sizeof(float)));
   ctx->recall_parts_cap = (int)((size_t)(ctx->num_sms + MAX_MT) * MAX_N * BM);
@@ -695,8 +694,8 @@ oda_status recall_setup(oda_ctx* ctx) {
   // the cluster split-K kernel: the largest cluster (8, 4, 2) the GPU holds
   ctx->recall_cluster_max = 0;
   const size_t csm = cl_smem_for(CL_MAX_N, cl_stages_for(CL_MAX_N));
-  if (cudaFuncSetAttribute(recall_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)csm) == cudaSuccess) {
+  if (raise_smem_limit(reinterpret_cast<const void*>(recall_cluster_kernel), csm) ==
+      cudaSuccess) {
     for (int ks = 8; ks >= 2; ks >>= 1) {
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(ks);

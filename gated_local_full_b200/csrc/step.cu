@@ -35,6 +35,14 @@ size_t layer_elems(const oda_ctx* ctx, int B, int heads) {
   return (size_t)B * heads * ctx->cfg.head_dim;
 }
 
+// Early staging (launch_attn's `early`): the append kernel writes the ring
+// and the paged cache of every layer, the record copy before it holds the
+// lengths, and the gate writes the compacted ids. Every Local launch after the
+// first follows another Local launch, and every Full launch after the first
+// another Full launch; none of them writes those inputs, and each waits for
+// its predecessor before it lets the next launch start. So from the second
+// launch of each kind on, the inputs a launch stages before its own
+// dependency wait were complete before it started.
 oda_status pre_part(oda_ctx* ctx, const oda_step_desc* d, cudaStream_t st,
                     unsigned long long cond, bool set_cond) {
   const oda_config& c = ctx->cfg;
@@ -48,7 +56,8 @@ oda_status pre_part(oda_ctx* ctx, const oda_step_desc* d, cudaStream_t st,
     float* lse = d->lse ? d->lse + (size_t)l * d->B * c.hq : nullptr;
     s = oda_impl::launch_attn(ctx, true, l, static_cast<const char*>(d->q) + qo, d->seq_lens,
                               d->ring, nullptr, nullptr, nullptr,
-                              static_cast<char*>(d->out) + qo, lse, d->B, st, ctx->plan_local);
+                              static_cast<char*>(d->out) + qo, lse, d->B, st, ctx->plan_local,
+                              /*early=*/l > 0);
     if (s != ODA_OK) return s;
   }
   if (d->W1) {
@@ -69,7 +78,8 @@ oda_status full_part(oda_ctx* ctx, const oda_step_desc* d, cudaStream_t st) {
     float* lse = d->lse ? d->lse + (size_t)l * d->B * c.hq : nullptr;
     oda_status s = oda_impl::launch_attn(ctx, false, l, static_cast<const char*>(d->q) + qo,
                                          d->seq_lens, d->kv_cache, d->block_table, d->idx,
-                                         d->count, static_cast<char*>(d->out) + qo, lse, d->B, st);
+                                         d->count, static_cast<char*>(d->out) + qo, lse, d->B, st,
+                                         nullptr, /*early=*/l > 0);
     if (s != ODA_OK) return s;
   }
   return ODA_OK;

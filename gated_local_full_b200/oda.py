@@ -22,6 +22,7 @@ LIB_PATH = os.path.join(_HERE, "liboda.so")
 OK, ERR_ARG, ERR_SHAPE, ERR_DTYPE, ERR_CUDA, ERR_TIMEOUT, ERR_BOUNDS, ERR_STATE = range(8)
 BF16, F32 = 0, 1
 MAX_BATCH = 1024
+ATTN_INPUTS_READY = 1     # oda_local_attn / oda_full_attn_gated flag (see oda.h)
 STATUS_NAMES = {0: "ODA_OK", 1: "ODA_ERR_ARG", 2: "ODA_ERR_SHAPE", 3: "ODA_ERR_DTYPE",
                 4: "ODA_ERR_CUDA", 5: "ODA_ERR_TIMEOUT", 6: "ODA_ERR_BOUNDS", 7: "ODA_ERR_STATE"}
 
@@ -84,11 +85,12 @@ def lib() -> ctypes.CDLL:
         "oda_destroy": [vp],
         "oda_append_kv": [vp, c_int, c_int, vp, vp, vp, vp, vp, vp, c_int, vp],
         "oda_ring_init": [vp, c_int, c_int, vp, vp, vp, vp, c_int, vp],
-        "oda_local_attn": [vp, c_int, vp, vp, vp, vp, vp, c_int, vp],
+        "oda_local_attn": [vp, c_int, vp, vp, vp, vp, vp, c_int, ctypes.c_uint, vp],
         "oda_recall_score": [vp, vp, vp, vp, c_int, vp, vp, vp, c_float, c_int, vp, c_int, vp],
         "oda_gate": [vp, vp, c_float, c_int, vp, vp, vp, vp],
         "oda_recall_loss": [vp, vp, vp, vp, c_float, c_int64, vp, vp, vp],
-        "oda_full_attn_gated": [vp, c_int, vp, vp, vp, vp, vp, vp, vp, vp, c_int, vp],
+        "oda_full_attn_gated": [vp, c_int, vp, vp, vp, vp, vp, vp, vp, vp, c_int, ctypes.c_uint,
+                                vp],
         "oda_get_device_error": [vp, vp, POINTER(c_int)],
         "oda_selftest_wait_timeout": [vp, c_uint64, vp],
         "oda_step_run": [vp, POINTER(OdaStepDesc), vp],
@@ -227,9 +229,14 @@ class OdaContext:
                                    ptr(block_table), ptr(kv_cache), ptr(ring), B,
                                    _stream(stream)), "oda_ring_init")
 
-    def local_attn(self, layer, q, seq_lens, ring, out, lse, B, stream=None):
+    def local_attn(self, layer, q, seq_lens, ring, out, lse, B, stream=None,
+                   inputs_ready=False):
+        """inputs_ready sets ODA_ATTN_INPUTS_READY (the ring and seq_lens were
+        complete before the previous kernel on the stream reached its wait)."""
         _check(lib().oda_local_attn(self.handle, layer, ptr(q), ptr(seq_lens), ptr(ring),
-                                    ptr(out), ptr(lse), B, _stream(stream)), "oda_local_attn")
+                                    ptr(out), ptr(lse), B,
+                                    ATTN_INPUTS_READY if inputs_ready else 0,
+                                    _stream(stream)), "oda_local_attn")
 
     def recall_score(self, h_prev, emb, h_local, H, W1, b1, w2, b2, hidden, scores, B,
                      stream=None):
@@ -251,11 +258,15 @@ class OdaContext:
                               ptr(count), _stream(stream)), "oda_gate")
 
     def full_attn_gated(self, layer, q, seq_lens, block_table, kv_cache, idx, count, out, lse,
-                        B, stream=None):
+                        B, stream=None, inputs_ready=False):
+        """inputs_ready sets ODA_ATTN_INPUTS_READY (cache, lengths, block table,
+        idx and count were complete before the previous kernel on the stream
+        reached its wait)."""
         _check(lib().oda_full_attn_gated(self.handle, layer, ptr(q), ptr(seq_lens),
                                          ptr(block_table), ptr(kv_cache), ptr(idx), ptr(count),
-                                         ptr(out), ptr(lse), B, _stream(stream)),
-               "oda_full_attn_gated")
+                                         ptr(out), ptr(lse), B,
+                                         ATTN_INPUTS_READY if inputs_ready else 0,
+                                         _stream(stream)), "oda_full_attn_gated")
 
     def get_device_error(self, stream=None) -> int:
         e = c_int(0)

@@ -42,7 +42,10 @@
  *     launches. Before the wait an attention kernel may read row ids,
  *     lengths and block-table entries (bypassing L1) only to choose which
  *     K/V lines to warm in L2 with bulk prefetches; these are read again
- *     after the wait, and a prefetch returns no value.
+ *     after the wait, and a prefetch returns no value. With the flag
+ *     ODA_ATTN_INPUTS_READY the caller states that those inputs and the K/V
+ *     were complete earlier, and the kernel also stages its first K/V tiles
+ *     before the wait (see that flag).
  */
 #ifndef ODA_H
 #define ODA_H
@@ -151,6 +154,24 @@ oda_status oda_ring_init(oda_ctx* ctx, int layer_begin, int layer_end,
                          const void* kv_cache, void* ring, int B, oda_stream stream);
 
 /*
+ * Flags of oda_local_attn and oda_full_attn_gated.
+ *
+ * ODA_ATTN_INPUTS_READY: the caller guarantees that the K/V source (ring or
+ * paged cache), seq_lens, block_table, idx and count of this call were
+ * complete before the previous kernel on `stream` reached its dependency wait
+ * -- for example because that kernel is another Local or Full launch of this
+ * library, which writes none of them and, like every kernel of this library,
+ * waits for its own predecessor before it lets the next launch start. The
+ * launch then works out its split and issues its first K/V tile copies into
+ * shared memory while the previous kernel is still running; it still reads
+ * the queries and writes its outputs and scratch only after that kernel has
+ * completed. Without the flag (0) the call makes no assumption beyond stream
+ * order. The captured step uses it for every Local and Full launch except the
+ * first of each kind.
+ */
+#define ODA_ATTN_INPUTS_READY 1u
+
+/*
  * Local attention F^L of one layer ([SUM] Methodology / Local-First Decoding):
  * for every row b and query head h,
  *   out[b][h] = sum_{j in S^L_t} softmax_j(q[b][h] . k_j / sqrt(d)) v_j,
@@ -164,10 +185,11 @@ oda_status oda_ring_init(oda_ctx* ctx, int layer_begin, int layer_end,
  * distributed shared memory; otherwise the split is merged through the
  * context's partials. The environment variable ODA_LOCAL_CLUSTER, read by
  * oda_create, caps the cluster size (0: always the partials merge).
+ * flags: 0 or ODA_ATTN_INPUTS_READY (see above); other bits: ODA_ERR_ARG.
  */
 oda_status oda_local_attn(oda_ctx* ctx, int layer, const void* q,
                           const int32_t* seq_lens, const void* ring,
-                          void* out, float* lse, int B, oda_stream stream);
+                          void* out, float* lse, int B, unsigned flags, oda_stream stream);
 
 /*
  * Recall score ([SUM] Methodology, q_t = R_psi(h_{t-1}, E(x_t), h^L_t)):
@@ -223,12 +245,13 @@ oda_status oda_gate(oda_ctx* ctx, const float* scores, float theta, int B,
  *   q, out       device [B][hq][d];  lse: device float [B][hq] or NULL
  *   kv_cache     paged cache of all layers;  idx, count: device (from oda_gate)
  * *count and idx are read on the device: no host synchronization.
+ * flags: 0 or ODA_ATTN_INPUTS_READY (see above); other bits: ODA_ERR_ARG.
  */
 oda_status oda_full_attn_gated(oda_ctx* ctx, int layer, const void* q,
                                const int32_t* seq_lens, const int32_t* block_table,
                                const void* kv_cache, const int32_t* idx,
                                const int32_t* count, void* out, float* lse, int B,
-                               oda_stream stream);
+                               unsigned flags, oda_stream stream);
 
 /*
  * Full attention for callers that cannot allocate device memory (the pages
@@ -236,8 +259,10 @@ oda_status oda_full_attn_gated(oda_ctx* ctx, int layer, const void* q,
  * hand the whole GPU to their own pool allocator at start-up cannot have a
  * library call cudaMalloc later (it fails once the pool holds the memory, or
  * breaks the pool's accounting), and a cudaMalloc on a latency-critical decode
- * loop synchronizes the device. This entry point computes exactly what
- * oda_full_attn_gated computes, with the same arguments, but needs no context
+ * loop synchronizes the device. This entry point computes the same function
+ * as oda_full_attn_gated, with the same arguments (less `flags`), within the
+ * attention tolerance (its persistent grid is capped at 512 CTAs, so its
+ * split of the sequence may differ from a context's), but needs no context
  * and allocates nothing: its split partials and tickets live in fixed
  * __device__ arrays inside liboda (1 MiB of partials, 512 segment tickets),
  * held by every GPU that loads the library until the process exits.

@@ -88,8 +88,8 @@ def test_null_context_and_pointers_rejected_without_gpu():
     assert L.oda_create(None, None) == oda.ERR_ARG
     assert L.oda_destroy(None) == oda.OK
     assert L.oda_append_kv(None, 0, 1, None, None, None, None, None, None, 1, None) == oda.ERR_ARG
-    assert L.oda_local_attn(None, 0, None, None, None, None, None, 1, None) == oda.ERR_ARG
-    assert L.oda_full_attn_gated(None, 0, None, None, None, None, None, None, None, None, 1,
+    assert L.oda_local_attn(None, 0, None, None, None, None, None, 1, 0, None) == oda.ERR_ARG
+    assert L.oda_full_attn_gated(None, 0, None, None, None, None, None, None, None, None, 1, 0,
                                  None) == oda.ERR_ARG
     assert L.oda_gate(None, None, 0.0, 1, None, None, None, None) == oda.ERR_ARG
     assert L.oda_recall_score(None, None, None, None, 64, None, None, None, 0.0, 128, None, 1,

@@ -290,3 +290,99 @@ def test_argument_errors(torch):
     # B == 0 is a valid no-op
     ctx.local_attn(0, dw.q[0, 0], seq, dw.ring, b["out"], None, 0)
     assert ctx.get_device_error() == 0
+
+
+@pytest.mark.parametrize("shape", ["cluster_b2", "partials_b40"])
+def test_inputs_ready_back_to_back(torch, shape):
+    """Local and Full launches of consecutive layers with ODA_ATTN_INPUTS_READY
+    on every launch but the first (the step's order): the later launches stage
+    their first K/V tiles before their dependency wait. Every row, every head
+    and every layer is compared with the oracle; batch 2 takes the cluster
+    merge, batch 40 the partials merge with the append kernel's plan-free
+    in-kernel partition."""
+    L = 4
+    if shape == "cluster_b2":
+        t0 = (9000, 2100)
+    else:
+        rng = np.random.default_rng(17)
+        t0 = tuple(int(x) for x in rng.integers(1, 6000, size=40))
+    B = len(t0)
+    scores = np.where(np.arange(B) % 3 == 0, 1.0, -1.0).astype(np.float32)
+    w = synth.custom("ready_" + shape, layers=L, hq=16, hkv=8, d=128, window=2048,
+                     t0=t0, fixed_scores=scores, steps=1)
+    ctx, dw = hx.setup(w)
+    seq = dw.seq_lens[0]
+    ctx.append_kv(0, L, dw.k_new[0], dw.v_new[0], seq, dw.block_table, dw.cache, dw.ring, B)
+    dt = dw.q.dtype
+    loc = torch.zeros((L, B, w.hq, w.d), dtype=dt, device="cuda")
+    lse_l = torch.zeros((L, B, w.hq), dtype=torch.float32, device="cuda")
+    for l in range(L):
+        ctx.local_attn(l, dw.q[0, l], seq, dw.ring, loc[l], lse_l[l], B, inputs_ready=l > 0)
+    flags = torch.empty(B, dtype=torch.uint8, device="cuda")
+    idx = torch.empty(B, dtype=torch.int32, device="cuda")
+    count = torch.empty(1, dtype=torch.int32, device="cuda")
+    ctx.gate(dw.scores[0], 0.0, B, flags, idx, count)
+    out = loc.clone()
+    lse_o = lse_l.clone()
+    for l in range(L):
+        ctx.full_attn_gated(l, dw.q[0, l], seq, dw.block_table, dw.cache, idx, count, out[l],
+                            lse_o[l], B, inputs_ready=l > 0)
+    torch.cuda.synchronize()
+    assert ctx.get_device_error() == 0
+    f_ref, _, _ = O.gate(scores, 0.0)
+    loc64, out64 = hx.to_f64(loc, w), hx.to_f64(out, w)
+    lsl, lso = lse_l.cpu().numpy().astype(np.float64), lse_o.cpu().numpy().astype(np.float64)
+    atol, rtol = hx.tol(w)
+    for l in range(L):
+        for r in range(B):
+            ref = hx.oracle_row(w, 0, l, r)
+            hx.assert_close(loc64[l, r], ref["local"], atol, rtol, f"local l{l} r{r}")
+            hx.assert_close(lsl[l, r], ref["lse_local"], 1e-4, 1e-5, f"lse local l{l} r{r}")
+            want, wl = (ref["full"], ref["lse_full"]) if f_ref[r] else (ref["local"],
+                                                                          ref["lse_local"])
+            hx.assert_close(out64[l, r], want, atol, rtol, f"final l{l} r{r}")
+            hx.assert_close(lso[l, r], wl, 1e-4, 1e-5, f"final lse l{l} r{r}")
+    # a flag bit the library does not define is refused
+    from gated_local_full_b200 import oda
+    st = oda.lib().oda_local_attn(ctx.handle, 0, oda.ptr(dw.q[0, 0]), oda.ptr(seq),
+                                  oda.ptr(dw.ring), oda.ptr(loc[0]), None, B, 2,
+                                  oda._stream(None))
+    assert st == oda.ERR_ARG
+
+
+def test_smem_limit_never_lowered(torch):
+    """A context sized for 32 rows keeps working after a second context and an
+    allocation-free call sized for 4 rows: a kernel's shared-memory limit is
+    one value per process, and the library only ever raises it."""
+    from gated_local_full_b200 import oda
+    w = synth.custom("smemlim", hq=16, hkv=8, d=128, window=256, t0=(3000, 500, 1200, 77),
+                     fixed_scores=(1.0, 1.0, -1.0, 1.0), batch=4)
+    ctx, dw = hx.setup(w, max_batch=32)
+    small_cfg = oda.make_config(layers=1, max_batch=4, hq=16, hkv=8, head_dim=128, sink=4,
+                                window=256, dtype="bf16", max_blocks_per_seq=dw.max_blocks,
+                                num_blocks=dw.num_blocks)
+    small = oda.OdaContext(small_cfg)
+    b = _bufs(torch, w)
+    seq = dw.seq_lens[0]
+    ctx.append_kv(0, 1, dw.k_new[0, 0], dw.v_new[0, 0], seq, dw.block_table, dw.cache,
+                  dw.ring, 4)
+    ctx.gate(dw.scores[0], 0.0, 4, b["flags"], b["idx"], b["count"])
+    scratch = torch.zeros((4, w.hq, w.d), dtype=torch.bfloat16, device="cuda")
+    oda.full_attn_gated_static(small_cfg, 0, dw.q[0, 0], seq, dw.block_table, dw.cache,
+                               b["idx"], b["count"], scratch, None, 4)
+    # the 32-row context after both smaller users
+    ctx.local_attn(0, dw.q[0, 0], seq, dw.ring, b["out"], b["lse"], 4)
+    local = b["out"].clone()
+    ctx.full_attn_gated(0, dw.q[0, 0], seq, dw.block_table, dw.cache, b["idx"], b["count"],
+                        b["out"], b["lse"], 4)
+    torch.cuda.synchronize()
+    assert ctx.get_device_error() == 0 and small.get_device_error() == 0
+    loc, out, st = hx.to_f64(local, w), hx.to_f64(b["out"], w), hx.to_f64(scratch, w)
+    for r in range(4):
+        ref = hx.oracle_row(w, 0, 0, r)
+        hx.assert_close(loc[r], ref["local"], *hx.tol(w), what=f"local row {r}")
+        want = ref["full"] if r != 2 else ref["local"]
+        hx.assert_close(out[r], want, *hx.tol(w), what=f"final row {r}")
+        if r != 2:
+            hx.assert_close(st[r], ref["full"], *hx.tol(w), what=f"static row {r}")
+    small.close()

@@ -1,4 +1,5 @@
-"""The allocation-free Full-attention entry point against the regular one.
+"""The allocation-free Full-attention entry point against the regular one
+and against the float64 oracle.
 
 oda_full_attn_gated_static exists for callers that cannot call cudaMalloc
 (engines whose device memory all belongs to their own pool allocator, decode
@@ -54,6 +55,13 @@ def test_static_entry_point_matches_regular_twice():
                         ref_lse.cpu().numpy().astype(np.float64), 1e-4, 1e-5, f"call {call} lse")
         # unflagged row 1 is left untouched by both
         assert torch.count_nonzero(got[1]) == 0
+        # and the flagged rows equal the float64 oracle's Full attention
+        g64 = got.to(torch.float64).cpu().numpy()
+        for r in (0, 2, 3):
+            want = hx.oracle_row(w, 0, layer, r)
+            hx.assert_close(g64[r], want["full"], atol, rtol, f"call {call} row {r} vs oracle")
+            hx.assert_close(got_lse[r].cpu().numpy().astype(np.float64), want["lse_full"],
+                            1e-4, 1e-5, f"call {call} row {r} lse vs oracle")
     # sizes beyond the fixed arrays are refused before any launch
     big = oda.make_config(layers=1, max_batch=128, hq=16, hkv=8, head_dim=128, sink=4,
                           window=256, dtype="bf16", max_blocks_per_seq=dw.max_blocks,
