@@ -124,12 +124,6 @@ struct Chunk<float> {
   }
 };
 
-// A query chunk from global memory (L2, issued at once: see ld_cg_v4), widened
-// where it is first needed.
-template <typename T>
-__device__ __forceinline__ uint4 q_chunk(const T* p) {
-  return ld_cg_v4(p);
-}
 
 // Bits [lo, hi) of a 16-bit tile mask whose bit 0 is slot `base`.
 __device__ __forceinline__ uint32_t range_bits(int lo, int hi, int base) {
@@ -399,9 +393,9 @@ attn_kernel(const AttnArgs a) {
   // Cluster mode: each rank owns G*D/cs output elements of the segment. A
   // rank merges its warps' states (or takes an empty one) and pushes, with
   // remote shared-memory stores, its accumulator for every element to the
-  // element's owner and each head's (m, l) to every rank. The barrier that
-  // every rank arrived at on entry is waited for first, so every target CTA
-  // has started.
+  // element's owner and each head's (m, l) to every rank. The caller has
+  // waited for the barrier every rank arrived at on entry, so every target
+  // CTA has started.
   auto cluster_push = [&](bool filled) {
     if constexpr (CL) {
       namespace cg = cooperative_groups;
@@ -409,7 +403,6 @@ attn_kernel(const AttnArgs a) {
       const int cs = a.cluster;
       const int rank = (int)cl.block_rank();
       const int per = (G * D) / cs;
-      cluster_wait();
       for (int o = tid; o < G * D; o += W * 32) {
         const int h = o / D, dd = o % D;
         float mt = -INFINITY, lt = 0.f, at = 0.f;
@@ -520,6 +513,25 @@ attn_kernel(const AttnArgs a) {
     }
   };
 
+  // A segment's queries (and, in cluster mode, its row's t) are read once per
+  // CTA by warp 0 into shared memory: one request per CTA instead of one per
+  // warp keeps the hot lines of q from queueing at their L2 slice. Cluster
+  // mode has one segment per CTA, loaded here while the first copies fly.
+  // The copies are asynchronous (cp.async, no registers held) and awaited by
+  // warp 0 after whatever the caller overlaps with them (cluster mode: the
+  // wait for every rank); a barrier of the caller's then publishes them.
+  auto load_q = [&](int row, int g, bool with_t) {   // warp 0: issue
+    const unsigned char* src = reinterpret_cast<const unsigned char*>(a.q) +
+                               ((long long)row * hq + g * G) * D * (long long)sizeof(T);
+    for (int c = lane; c < QCH; c += 32) cp_async16(smem_addr(sq + c), src + 16 * c);
+    if (with_t && lane == 0) cp_async4(smem_addr(st_t), a.seq_lens + row);
+  };
+  auto store_q = [&](bool) {                         // warp 0: the copies have landed
+    cp_async_wait_all();
+  };
+  // Without early staging the first segment's queries are requested before
+  // the first tile copies, so they do not queue behind them.
+  bool q_loaded = false;
   int issued = 0;
   bool prod_done = false;
   if (has_work) {
@@ -539,6 +551,10 @@ attn_kernel(const AttnArgs a) {
     }
     use_pool = pool0 < seg_nt;
     q0 = q1 = seg_nt;
+    if (!early) {
+      if (warp == 0) load_q(seg_b, seg_g0, CL);
+      q_loaded = true;
+    }
     if (!CL && early && tid == 0)
       // the first segment's queries into L2 (a prefetch returns no value)
       bulk_prefetch_l2(reinterpret_cast<const T*>(a.q) +
@@ -563,23 +579,16 @@ attn_kernel(const AttnArgs a) {
   // (cluster mode never leaves early: every CTA takes part in the merge)
   if (!CL && !has_work) return;
   if (CL && !has_work) {
+    cluster_wait();                              // every rank has started
     cluster_push(false);                         // an empty state: m = -inf, l = acc = 0
   } else {
 
-  // A segment's queries (and, in cluster mode, its row's t) are read once per
-  // CTA by warp 0 into shared memory: one request per CTA instead of one per
-  // warp keeps the hot lines of q from queueing at their L2 slice. Cluster
-  // mode has one segment per CTA, loaded here while the first copies fly.
-  auto load_q = [&](int row, int g, bool with_t) {   // warp 0; the caller syncs
-    const unsigned char* src = reinterpret_cast<const unsigned char*>(a.q) +
-                               ((long long)row * hq + g * G) * D * (long long)sizeof(T);
-    for (int c = lane; c < QCH; c += 32) sq[c] = q_chunk(reinterpret_cast<const T*>(src + 16 * c));
-    if (with_t && lane == 0) st_t[0] = ld_cg_s32(a.seq_lens + row);
-  };
   uint4 qraw[G];
   int tpre = 0;
   if constexpr (CL) {
-    if (warp == 0) load_q(seg_b, seg_g0, true);
+    if (warp == 0 && !q_loaded) load_q(seg_b, seg_g0, true);
+    cluster_wait();                              // every rank has started (overlaps the loads)
+    if (warp == 0) store_q(true);
     __syncthreads();
 #pragma unroll
     for (int h = 0; h < G; ++h) qraw[h] = sq[h * LPR + li];
@@ -615,7 +624,11 @@ attn_kernel(const AttnArgs a) {
     // this lane's DPL dims of the G query heads (exact, unscaled)
     float2 q2[G][DP2];
     if constexpr (!CL) {
-      if (warp == 0) load_q(b, seg.g, false);
+      if (warp == 0) {
+        if (!q_loaded) load_q(b, seg.g, false);   // else requested with the first copies
+        store_q(false);
+      }
+      q_loaded = false;
       __syncthreads();
 #pragma unroll
       for (int h = 0; h < G; ++h) qraw[h] = sq[h * LPR + li];
@@ -1073,26 +1086,32 @@ attn_kernel(const AttnArgs a) {
     const int b = rowb[0], g = ((int)blockIdx.x / cs) % a.hkv;
     const float2* ml = reinterpret_cast<const float2*>(rml);
     T* outp = reinterpret_cast<T*>(a.out);
-    for (int ol = tid; ol < per; ol += W * 32) {
+    // cs consecutive lanes combine one owned element: lane r of the group
+    // takes rank r's (m, l, acc), and xor shuffles within the group (cs
+    // divides 32) give the maximum and the rescaled sums in a fixed order.
+    // per * cs = G * D is a multiple of 32, so a warp is wholly in or out.
+    for (int base = 0; base < per * cs; base += W * 32) {
+      const int it = base + tid;
+      if (it >= per * cs) break;
+      const int ol = it / cs, r = it % cs;
       const int o = rank * per + ol;
       const int h = o / D, dd = o % D;
-      float mt = -INFINITY;
-      for (int r = 0; r < cs; ++r) mt = fmaxf(mt, ml[r * G + h].x);
-      float lt = 0.f, at = 0.f;
-      if (mt != -INFINITY) {
-        for (int r = 0; r < cs; ++r) {
-          const float2 v = ml[r * G + h];
-          if (v.x == -INFINITY) continue;
-          const float sc2 = fast_exp2(v.x - mt);
-          lt += v.y * sc2;
-          at += racc[r * per + ol] * sc2;
-        }
+      const float2 v = ml[r * G + h];
+      float mt = v.x;
+      for (int x = 1; x < cs; x <<= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, x));
+      const float sc2 = (v.x == -INFINITY) ? 0.f : fast_exp2(v.x - mt);
+      float lt = v.y * sc2, at = racc[r * per + ol] * sc2;
+      for (int x = 1; x < cs; x <<= 1) {
+        lt += __shfl_xor_sync(0xffffffffu, lt, x);
+        at += __shfl_xor_sync(0xffffffffu, at, x);
       }
-      const long long orow = ((long long)b * hq + g * G + h) * D;
-      outp[orow + dd] = (T)(lt > 0.f ? at / lt : 0.f);
-      if (dd == 0 && a.lse)
-        a.lse[(long long)b * hq + g * G + h] =
-            lt > 0.f ? (mt + fast_log2(lt)) * 0.69314718055994531f : -INFINITY;
+      if (r == 0) {
+        const long long orow = ((long long)b * hq + g * G + h) * D;
+        outp[orow + dd] = (T)(lt > 0.f ? at / lt : 0.f);
+        if (dd == 0 && a.lse)
+          a.lse[(long long)b * hq + g * G + h] =
+              lt > 0.f ? (mt + fast_log2(lt)) * 0.69314718055994531f : -INFINITY;
+      }
     }
   }
 }
@@ -1208,6 +1227,7 @@ template <typename T, int D, int G, int W, int NS>
 oda_status launch_cluster(oda_ctx* ctx, const AttnArgs& a, int grid, int cs, cudaStream_t st) {
   auto k = attn_kernel<T, D, G, W, NS, true, true>;
   const size_t sm = smem_bytes_wn<T, D, G, W, NS>(ctx->cfg.max_batch);
+  ctx->local_last_smem = sm;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(W * 32);
@@ -1229,6 +1249,7 @@ template <typename T, int D, int G, bool RING>
 oda_status launch_one(oda_ctx* ctx, const AttnArgs& a, int ctas, cudaStream_t st) {
   auto k = kernel_ptr<T, D, G, RING>();
   const size_t sm = smem_bytes<T, D, G, RING>(ctx->cfg.max_batch);
+  if (RING) ctx->local_last_smem = sm;
   return launch_pdl(k, dim3(ctas), dim3(Shape<T, D, G>::W * 32), sm, st, a) == cudaSuccess
              ? ODA_OK
              : ODA_ERR_CUDA;

@@ -32,6 +32,18 @@ struct oda_ctx {
   int local_cluster_max;     // largest cluster for the cluster-merge Local kernel (0: none)
   int local_wide_cluster_max;  // the same for its one-tile-per-warp shape
   int local_wide_ctas;       // CTAs of that shape one wave holds
+  size_t local_last_smem;    // dynamic shared memory of the last Local launch issued
+};
+
+// The gate run by the recall head's last CTA inside a captured step.
+struct RecallGate {
+  const float* scores;       // scores to compare; null: the head's own output
+  float theta;
+  uint8_t* flags;
+  int32_t* idx;
+  int32_t* count;
+  unsigned long long cond;   // conditional-node handle
+  bool set_cond;
 };
 
 namespace oda {
@@ -165,21 +177,16 @@ __device__ __forceinline__ float fast_log2(float x) {
   return y;
 }
 
-// 16-byte global load through L2 only (bypassing L1), issued where it stands:
-// the asm is volatile, so the compiler neither drops nor sinks it below later
-// volatile operations (a load whose result is needed late still leaves early).
-__device__ __forceinline__ uint4 ld_cg_v4(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
+// Asynchronous global -> shared copies that hold no registers (cp.async):
+// 16 bytes through L2 only, or 4 bytes; wait_all waits for this thread's.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
-
-__device__ __forceinline__ int ld_cg_s32(const int* p) {
-  int v;
-  asm volatile("ld.global.cg.s32 %0, [%1];" : "=r"(v) : "l"(p));
-  return v;
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
 // bf16 pair (packed in a 32-bit word, low half first) -> two floats, exactly.
@@ -237,7 +244,8 @@ oda_status launch_gate(oda_ctx* ctx, const float* scores, float theta, int B, ui
                        unsigned long long cond_handle, bool set_cond);
 oda_status launch_recall(oda_ctx* ctx, const void* h_prev, const void* emb, const void* h_local,
                          int H, const void* W1, const float* b1, const float* w2, float b2,
-                         int hidden, float* scores, int B, cudaStream_t st);
+                         int hidden, float* scores, int B, cudaStream_t st, bool early = false,
+                         const RecallGate* gate = nullptr, bool* gate_fused = nullptr);
 oda_status recall_setup(oda_ctx* ctx);
 oda_status launch_recall_loss(oda_ctx* ctx, const float* q, const float* lpf, const float* lpl,
                               float lam, long long n, float* loss, int32_t* n_full,

@@ -27,6 +27,7 @@
 #include <cooperative_groups.h>
 #include <cuda.h>
 
+#include "gate.cuh"
 #include "oda_internal.cuh"
 
 using namespace oda;
@@ -50,6 +51,17 @@ struct RecallArgs {
   int* tickets;      // [MT] per m-tile, [MAX_MT] for the final sum
   int* err;
   int B, N, MT, KB, H, stages;
+  // Cluster kernel only: stage the first W1 tiles before the dependency wait
+  // (the weights were written before the previous kernel started), and gate
+  // the scores in the last CTA (gate_scores non-null).
+  int early;
+  const float* gate_scores;     // the scores the gate compares (the head's own or given)
+  float theta;
+  uint8_t* flags;
+  int32_t* idx;
+  int32_t* count;
+  unsigned long long cond;      // conditional-node handle set from the count, if set_cond
+  int set_cond;
 };
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
@@ -453,6 +465,13 @@ recall_cluster_kernel(const __grid_constant__ CUtensorMap tm_w1,
   while ((int)ncols < N) ncols <<= 1;
 
   cluster_arrive_relaxed();                               // "started": waited for before any push
+  // Early mode: the first stages' W1 tiles are requested before the
+  // dependency wait (each stage's barrier expects the W1 and the state tile;
+  // the state tile, which a preceding kernel may write, follows after the
+  // wait). The owner rows' b1 and w2 are read with them.
+  const int pre = a.early ? min(S, kb1 - kb0) : 0;
+  float* sb1 = red + 192;                                 // [RP] b1 of the owned rows
+  float* sw2 = sb1 + BM;                                  // [RP] w2 of the owned rows
   if (tid == 0) {
     for (int s2 = 0; s2 < S; ++s2) {
       mbar_init(smem_addr(&full[s2]), 1);
@@ -460,9 +479,24 @@ recall_cluster_kernel(const __grid_constant__ CUtensorMap tm_w1,
     }
     mbar_init(smem_addr(acc_full), 1);
     fence_mbar_init();
+    const uint32_t tx = A_STAGE_BYTES + b_stage_bytes;
+    for (int i = 0; i < pre; ++i) {
+      const uint32_t fb = smem_addr(&full[i]);
+      mbar_arrive_expect_tx(fb, tx);
+      tma_load_2d(smem_addr(sa + (size_t)i * A_STAGE_BYTES), &tm_w1, (kb0 + i) * BK, mt * BM, fb);
+    }
   }
+  auto load_owner_weights = [&]() {
+    for (int rl = tid - 64; rl >= 0 && rl < RP; rl += 128) {
+      const int row = mt * BM + rank * RP + rl;
+      sb1[rl] = a.b1[row];
+      sw2[rl] = a.w2[row];
+    }
+  };
+  if (a.early && warp >= 2) load_owner_weights();
   pdl_wait();
   pdl_launch_dependents();
+  if (!a.early && warp >= 2) load_owner_weights();
   if (warp == 0) {
     __syncwarp();
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -482,14 +516,16 @@ recall_cluster_kernel(const __grid_constant__ CUtensorMap tm_w1,
       const uint32_t tx = A_STAGE_BYTES + b_stage_bytes;
       for (int kb = kb0, i = 0; kb < kb1; ++kb, ++i) {
         const int s2 = i % S;
-        const uint32_t par = (uint32_t)(((i / S) & 1) ^ 1);
-        if (!mbar_wait_bounded(smem_addr(&empty[s2]), par, kWaitLimitNs)) {
-          record_error(a.err, ODA_ERR_TIMEOUT);
-          break;
-        }
         const uint32_t fb = smem_addr(&full[s2]);
-        mbar_arrive_expect_tx(fb, tx);
-        tma_load_2d(smem_addr(sa + (size_t)s2 * A_STAGE_BYTES), &tm_w1, kb * BK, mt * BM, fb);
+        if (i >= pre) {                                   // else W1 was requested early
+          const uint32_t par = (uint32_t)(((i / S) & 1) ^ 1);
+          if (!mbar_wait_bounded(smem_addr(&empty[s2]), par, kWaitLimitNs)) {
+            record_error(a.err, ODA_ERR_TIMEOUT);
+            break;
+          }
+          mbar_arrive_expect_tx(fb, tx);
+          tma_load_2d(smem_addr(sa + (size_t)s2 * A_STAGE_BYTES), &tm_w1, kb * BK, mt * BM, fb);
+        }
         const int kglob = kb * BK;
         const int seg = kglob / a.H;
         const int kin = kglob - seg * a.H;
@@ -563,8 +599,7 @@ recall_cluster_kernel(const __grid_constant__ CUtensorMap tm_w1,
     for (int rl = t0; rl < RP; rl += TPN) {               // fixed order
       float u = 0.f;
       for (int r2 = 0; r2 < KS; ++r2) u += rbuf[((size_t)r2 * RP + rl) * N + n];
-      const int row = mt * BM + rank * RP + rl;
-      s += a.w2[row] * gelu_erf(u + a.b1[row]);
+      s += sw2[rl] * gelu_erf(u + sb1[rl]);
     }
     red[j] = s;
   }
@@ -591,9 +626,25 @@ recall_cluster_kernel(const __grid_constant__ CUtensorMap tm_w1,
     // grp, grp + ngrp, ... of batch row n; the groups are then added in order
     const int ngrp = 192 / a.B;                           // B <= 64: at least 3 groups
     const int n = tid % a.B, grp = tid / a.B;
+    // With at most 32 rows warp 0 gates alone; scores given to the gate from
+    // outside are requested together with the partials.
+    const bool warp_gate = a.gate_scores != nullptr && a.B <= 32;
+    const bool own = a.gate_scores == a.scores;
+    float gval = 0.f;
+    if (warp_gate && !own && tid < a.B) gval = __ldcg(a.gate_scores + tid);
     float v = 0.f;
     if (grp < ngrp) {
-      for (int c2 = grp; c2 < (int)gridDim.x; c2 += ngrp) v += __ldcg(a.spart + (size_t)c2 * N + n);
+      // eight partials requested at a time, added in CTA order
+      for (int c2 = grp; c2 < (int)gridDim.x; c2 += 8 * ngrp) {
+        float x[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int cc = c2 + u * ngrp;
+          x[u] = cc < (int)gridDim.x ? __ldcg(a.spart + (size_t)cc * N + n) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v += x[u];
+      }
       red[grp * a.B + n] = v;
     }
     __syncthreads();
@@ -601,8 +652,18 @@ recall_cluster_kernel(const __grid_constant__ CUtensorMap tm_w1,
       float t2 = 0.f;
       for (int g2 = 0; g2 < ngrp; ++g2) t2 += red[g2 * a.B + tid];
       a.scores[tid] = t2 + a.b2;
+      if (warp_gate && own) gval = t2 + a.b2;
     }
     if (tid == 0) a.tickets[MAX_MT] = 0;
+    if (warp_gate) {
+      if (warp == 0)
+        gate_warp(gval, a.B, a.theta, a.flags, a.idx, a.count, (cudaGraphConditionalHandle)a.cond,
+                  a.set_cond);
+    } else if (a.gate_scores) {
+      __syncthreads();                                    // the scores above are visible
+      gate_block(a.gate_scores, a.theta, a.B, a.flags, a.idx, a.count,
+                 (cudaGraphConditionalHandle)a.cond, a.set_cond, reinterpret_cast<int*>(red));
+    }
   }
   __syncthreads();
   if (warp == 0) {
@@ -674,7 +735,14 @@ int cl_stages_for(int n) {
 
 size_t cl_smem_for(int n, int s) {
   return 1024 + (size_t)s * (A_STAGE_BYTES + n * BK * 2) + (size_t)(2 * s + 1) * 8 + 4 + 16 + 16 +
-         (size_t)(BM * n + 192) * 4 + 64;
+         (size_t)(BM * n + 192 + 2 * BM) * 4 + 64;
+}
+
+// Stages of the cluster kernel within `budget` bytes of shared memory.
+int cl_stages_within(int n, size_t budget) {
+  int s = 8;
+  while (s > 2 && cl_smem_for(n, s) > budget) --s;
+  return s;
 }
 
 }  // namespace
@@ -722,7 +790,9 @@ oda_status recall_setup(oda_ctx* ctx) {
 
 oda_status launch_recall(oda_ctx* ctx, const void* h_prev, const void* emb, const void* h_local,
                          int H, const void* W1, const float* b1, const float* w2, float b2,
-                         int hidden, float* scores, int B, cudaStream_t st) {
+                         int hidden, float* scores, int B, cudaStream_t st, bool early,
+                         const RecallGate* gate, bool* gate_fused) {
+  if (gate_fused) *gate_fused = false;
   if (B < 1 || B > MAX_N || H < BK || H % BK != 0 || hidden < BM || hidden % BM != 0 ||
       hidden / BM > MAX_MT)
     return ODA_ERR_SHAPE;
@@ -747,6 +817,14 @@ oda_status launch_recall(oda_ctx* ctx, const void* h_prev, const void* emb, cons
   a.MT = hidden / BM;
   a.KB = (int)(K / BK);
   a.H = H;
+  a.early = 0;
+  a.gate_scores = nullptr;
+  a.theta = 0.f;
+  a.flags = nullptr;
+  a.idx = nullptr;
+  a.count = nullptr;
+  a.cond = 0ull;
+  a.set_cond = 0;
   // cluster split-K when every m-tile gets a whole cluster within one wave
   int KS = 0;
   if (N == 16 || N == 32 || N == 64) {
@@ -755,6 +833,25 @@ oda_status launch_recall(oda_ctx* ctx, const void* h_prev, const void* emb, cons
   }
   if (KS >= 2) {
     a.stages = cl_stages_for(N);
+    if (early) {
+      // The CTAs are to become resident beside the preceding Local launch's
+      // CTAs (one per SM) and request W1 while it runs: fewer stages, so both
+      // fit one SM's shared memory (1 KB of it is reserved per CTA).
+      const size_t sm_total = 228 * 1024;
+      const size_t beside = ctx->local_last_smem + 2 * 1024;
+      if (ctx->local_last_smem > 0 && beside + cl_smem_for(N, 2) <= sm_total)
+        a.stages = cl_stages_within(N, sm_total - beside);
+      a.early = 1;
+    }
+    if (gate && B <= 192) {
+      a.gate_scores = gate->scores ? gate->scores : scores;
+      a.theta = gate->theta;
+      a.flags = gate->flags;
+      a.idx = gate->idx;
+      a.count = gate->count;
+      a.cond = gate->cond;
+      a.set_cond = gate->set_cond ? 1 : 0;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(a.MT * KS);
     cfg.blockDim = dim3(192);
@@ -769,9 +866,10 @@ oda_status launch_recall(oda_ctx* ctx, const void* h_prev, const void* emb, cons
     at[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = at;
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, recall_cluster_kernel, tw, t0, t1, t2, a, KS) == cudaSuccess
-               ? ODA_OK
-               : ODA_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, recall_cluster_kernel, tw, t0, t1, t2, a, KS) != cudaSuccess)
+      return ODA_ERR_CUDA;
+    if (gate_fused) *gate_fused = a.gate_scores != nullptr;
+    return ODA_OK;
   }
   a.stages = stages_for(N);
   const int U = a.MT * a.KB;

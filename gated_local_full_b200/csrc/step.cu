@@ -60,12 +60,25 @@ oda_status pre_part(oda_ctx* ctx, const oda_step_desc* d, cudaStream_t st,
                               /*early=*/l > 0);
     if (s != ODA_OK) return s;
   }
+  const float* gs = d->gate_scores ? d->gate_scores : d->scores;
+  bool gated = false;
   if (d->W1) {
+    // The recall head follows the last Local launch, which writes none of its
+    // weights: it requests its first W1 tiles before its dependency wait, and
+    // its last CTA gates the scores, so the step needs no gate launch.
+    RecallGate g;
+    g.scores = gs;
+    g.theta = d->theta;
+    g.flags = d->flags;
+    g.idx = d->idx;
+    g.count = d->count;
+    g.cond = cond;
+    g.set_cond = set_cond;
     s = oda_impl::launch_recall(ctx, d->h_prev, d->emb, d->h_local, d->H, d->W1, d->b1, d->w2,
-                                d->b2, d->hidden, d->scores, d->B, st);
+                                d->b2, d->hidden, d->scores, d->B, st, /*early=*/true, &g, &gated);
     if (s != ODA_OK) return s;
   }
-  const float* gs = d->gate_scores ? d->gate_scores : d->scores;
+  if (gated) return ODA_OK;
   return oda_impl::launch_gate(ctx, gs, d->theta, d->B, d->flags, d->idx, d->count, st, cond,
                                set_cond);
 }

@@ -299,13 +299,14 @@ def tiny_fp32() -> Workload:
     return w
 
 
-def ctx16k(batch: int = 8) -> Workload:
+def ctx16k(batch: int = 8, steps: int = 1) -> Workload:
     """bf16, 1 layer, batch 8, 16/8 heads, d=128, every context 16384, paged
     block 16, K/V ~ N(0,1)*0.5, flags Bernoulli(0.41) per row, one needle per
-    flagged row."""
+    flagged row. `steps` > 1 continues the same requests (t grows by one per
+    step)."""
     w = Workload(name="ctx16k_b8", dtype="bf16", layers=1, batch=batch, hq=16, hkv=8, d=128,
                  sink=4, window=2048, block_size=16,
-                 t0=np.full(batch, 16384, np.int64), steps=1, seed=1,
+                 t0=np.full(batch, 16384, np.int64), steps=steps, seed=1,
                  flag_rate=0.41, flag_per="row", needles_on=True)
     f = w.flags()[0]
     _plant_needles(w, [b for b in range(batch) if f[b]])
@@ -328,7 +329,7 @@ def ctx128k(steps: int = 1024, layers: int = 28, context: int = 131072,
 MIXED_RATES = (0.0, 0.125, 0.41, 1.0)
 
 
-def mixed_batch(rate: float, batch: int = 32) -> Workload:
+def mixed_batch(rate: float, batch: int = 32, steps: int = 1) -> Workload:
     """bf16, batch 32, contexts uniform in [4096, 65536], 16/8 heads, d=128,
     paged block 16, Full calls Bernoulli(rate) per row, append inside the step."""
     rng = np.random.Generator(np.random.PCG64([3, 7004]))
@@ -336,16 +337,16 @@ def mixed_batch(rate: float, batch: int = 32) -> Workload:
     sub = MIXED_RATES.index(rate) if rate in MIXED_RATES else 99
     return Workload(name=f"mixed_b{batch}_rho{rate:g}", dtype="bf16", layers=1, batch=batch,
                     hq=16, hkv=8, d=128, sink=4, window=2048, block_size=16, t0=t0,
-                    steps=1, seed=3 * 1000 + sub, flag_rate=rate, flag_per="row")
+                    steps=steps, seed=3 * 1000 + sub, flag_rate=rate, flag_per="row")
 
 
-def recall_step(ctx: int, batch: int = 16) -> Workload:
+def recall_step(ctx: int, batch: int = 16, steps: int = 1) -> Workload:
     """bf16, batch 16, hidden 2048, recall MLP 6144 -> 4096 -> 1 (GELU),
     Xavier-uniform weights, N(0,1) hidden states, theta = 0, 16/8 heads, d=128,
     every context ``ctx`` (4096 or 131072)."""
     return Workload(name=f"recall_b{batch}_ctx{ctx}", dtype="bf16", layers=1, batch=batch,
                     hq=16, hkv=8, d=128, sink=4, window=2048, block_size=16,
-                    t0=np.full(batch, ctx, np.int64), steps=1, seed=4, recall=True)
+                    t0=np.full(batch, ctx, np.int64), steps=steps, seed=4, recall=True)
 
 
 def custom(name: str, *, dtype="bf16", layers=1, batch=None, hq=4, hkv=2, d=128, sink=4,

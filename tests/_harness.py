@@ -116,3 +116,25 @@ def oracle_head(w: Workload, q_row: np.ndarray, layer: int, row: int, g: int, t:
         return O.full_attention(q, K, V, t)
     K, V = oracle_kv_head(w, layer, row, g, t, O.local_access_set(t, w.sink, w.window))
     return O.local_attention(q, K, V, t, w.sink, w.window)
+
+
+def _head_task(args):
+    """One oracle (layer, row, KV head) evaluation in a worker process."""
+    w, q_row, layer, row, g, t, full = args
+    return oracle_head(w, q_row, layer, row, g, t, full)
+
+
+def oracle_heads(w: Workload, tasks, workers=None):
+    """Oracle outputs for many (q_row [hq][d], layer, row, kv_head, t, full)
+    tasks, in order: [(out [G][d], lse [G]), ...]. Generating a long row's
+    K/V dominates, so the tasks run in a pool of processes started with
+    spawn (safe beside a CUDA context); small task lists run inline."""
+    import concurrent.futures as cf
+    import multiprocessing as mp
+    import os
+    args = [(w, q, l, b, g, t, f) for (q, l, b, g, t, f) in tasks]
+    n = workers or min(len(os.sched_getaffinity(0)), 16)
+    if len(args) <= 2 or n <= 1:
+        return [_head_task(a) for a in args]
+    with cf.ProcessPoolExecutor(max_workers=n, mp_context=mp.get_context("spawn")) as ex:
+        return list(ex.map(_head_task, args, chunksize=1))

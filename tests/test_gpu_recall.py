@@ -124,11 +124,12 @@ def test_gated_step_with_recall_head(torch, ctxlen):
     # attention: sampled rows and heads (all rows' Local at ctx 4096)
     out = hx.to_f64(st.out[0], w)
     q = w.q_step(0)[0]
-    rows = range(w.batch) if ctxlen <= 4096 else [int(np.argmax(flags)), int(np.argmin(flags))]
+    # every row; two KV heads each at 131072, all eight at 4096
     rng = np.random.default_rng(ctxlen)
-    for b in rows:
-        g = int(rng.integers(0, w.hkv))
-        o, _ = hx.oracle_head(w, q[b], 0, b, g, ctxlen, full=bool(flags[b]))
+    pairs = [(b, g) for b in range(w.batch) for g in
+             (range(w.hkv) if ctxlen <= 4096 else rng.choice(w.hkv, 2, replace=False))]
+    tasks = [(q[b], 0, b, int(g), ctxlen, bool(flags[b])) for (b, g) in pairs]
+    for (b, g), (o, _) in zip(pairs, hx.oracle_heads(w, tasks)):
         hx.assert_close(out[b, g * w.group:(g + 1) * w.group], o, *hx.tol(w),
                         what=f"row {b} head {g}")
     st.close()

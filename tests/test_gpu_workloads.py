@@ -21,43 +21,52 @@ def torch():
 
 
 def _check_heads(w, out_step, q_step, step, pairs, flags_row):
-    """out_step: [L][B][hq][d] float64; pairs: (layer, row, kv_head)."""
-    for (l, b, g) in pairs:
-        t = int(w.t0[b]) + step
-        o, _ = hx.oracle_head(w, q_step[l, b], l, b, g, t, full=bool(flags_row[b]))
+    """out_step: [L][B][hq][d] float64; pairs: (layer, row, kv_head). The
+    oracle evaluations run in a process pool (see hx.oracle_heads)."""
+    tasks = [(q_step[l, b], l, b, g, int(w.t0[b]) + step, bool(flags_row[b])) for (l, b, g) in pairs]
+    for (l, b, g), (o, _) in zip(pairs, hx.oracle_heads(w, tasks)):
         hx.assert_close(out_step[l, b, g * w.group:(g + 1) * w.group], o, *hx.tol(w),
                         what=f"step {step} layer {l} row {b} head {g}")
 
 
 def test_ctx128k_graph_sampled(torch):
-    """batch 1, 28 layers, t = 131072 + step, Full calls drawn per step:
-    steps 0..6 run through the captured step graph; an unflagged step (1)
-    and two flagged steps (2, 6) are checked on sampled (layer, head) pairs."""
+    """batch 1, 28 layers, t = 131072 + step, Full calls drawn per step, with
+    the recall head in the step (its last CTA gates the injected scores):
+    steps 0..7 run through the captured step graph. Every flagged step is
+    checked on all 8 KV heads of layers 0 and 27; an unflagged step the
+    same; and 16 random (step, layer, head) triples besides."""
     from gated_local_full_b200.runtime import DecodeStep
-    w = synth.ctx128k(steps=7)
+    w = synth.ctx128k(steps=8)
+    w.recall = True
     flags = w.flags()[:, 0]
     assert flags[1] == 0 and flags[2] == 1 and flags[6] == 1
     ctx, dw = hx.setup(w)
-    st = DecodeStep(ctx, 1, dw.cache, dw.ring, dw.block_table, external_scores=True,
+    r = dw.recall
+    st = DecodeStep(ctx, 1, dw.cache, dw.ring, dw.block_table, recall=r, external_scores=True,
                     with_lse=True)
     keep = {}
     for step in range(w.steps):
         st.feed(dw.q[step], dw.k_new[step], dw.v_new[step], dw.seq_lens[step],
-                gate_scores=dw.scores[step])
+                gate_scores=dw.scores[step], h_prev=r["h_prev"][step], emb=r["emb"][step],
+                h_local=r["h_local"][step])
         st.run()
-        if step in (1, 2, 6):
-            keep[step] = (st.out.to(torch.float64).cpu().numpy(), int(st.count.item()),
-                          st.flags.cpu().numpy().copy())
+        keep[step] = (st.out.to(torch.float64).cpu().numpy(), int(st.count.item()),
+                      st.flags.cpu().numpy().copy())
     torch.cuda.synchronize()
     assert ctx.get_device_error() == 0
     rng = np.random.default_rng(5)
-    for step in (1, 2, 6):
+    extra = {}
+    for _ in range(16):
+        s_, l_, g_ = int(rng.integers(0, w.steps)), int(rng.integers(1, 27)), int(rng.integers(0, 8))
+        extra.setdefault(s_, []).append((l_, 0, g_))
+    checked = [i for i in range(w.steps) if flags[i]] + [1]
+    for step in range(w.steps):
         out, count, fl = keep[step]
         assert count == int(flags[step]) and fl[0] == flags[step]
-        q = w.q_step(step)
-        pairs = [(0, 0, 0), (27, 0, 7)] + [(int(rng.integers(1, 27)), 0, int(rng.integers(0, 8)))
-                                           for _ in range(2 if step != 1 else 1)]
-        _check_heads(w, out, q, step, pairs, fl)
+        pairs = ([(l, 0, g) for l in (0, 27) for g in range(8)] if step in checked else [])
+        pairs += extra.get(step, [])
+        if pairs:
+            _check_heads(w, out, w.q_step(step), step, pairs, fl)
     st.close()
 
 
@@ -79,11 +88,8 @@ def test_mixed_batch(torch, rate):
     assert st.idx.cpu().numpy().tolist() == i.tolist() and int(st.count.item()) == c
     out = st.out.to(torch.float64).cpu().numpy()
     q = w.q_step(0)
-    rng = np.random.default_rng(int(rate * 1000))
-    flagged = [b for b in range(w.batch) if flags[b]]
-    # Local for every row (one sampled head each), Full for up to 3 flagged rows
-    pairs = [(0, b, int(rng.integers(0, w.hkv))) for b in range(w.batch) if not flags[b]]
-    pairs += [(0, b, int(rng.integers(0, w.hkv))) for b in flagged[:3]]
+    # every row and every KV head: Full for the flagged rows, Local for the rest
+    pairs = [(0, b, g) for b in range(w.batch) for g in range(w.hkv)]
     _check_heads(w, out, q, 0, pairs, flags)
     st.close()
 
