@@ -1,16 +1,26 @@
 #!/usr/bin/env python
 """Benchmark of the gated local/full decode-attention step on B200.
 
-Workload (default): batch 1, 28 layers of GQA attention (16 query / 8 KV
-heads, head_dim 128, bf16), context t = 131072 at the first step and growing
-by one per step, s = 4 sinks + w = 2048 window for Local, Full recomputation
-on a Bernoulli(0.125) draw per step, plus the 6144 -> 4096 -> 1 recall head
-on synthetic states every step. One "step" = one decode step of the whole
-path (append, Local x 28, recall head, gate, Full x 28 when flagged) replayed
-from a captured CUDA graph; inputs are resident in HBM and fed with one
-device copy per step.
+Workloads (--workload):
+  ctx128k (default, the headline): batch 1, 28 layers of GQA attention (16
+      query / 8 KV heads, head_dim 128, bf16), context t = 131072 at the first
+      step and growing by one per step, s = 4 sinks + w = 2048 window for
+      Local, Full recomputation on a Bernoulli(0.125) draw per step;
+  ctx16k: batch 8, one layer, t = 16384, Full calls Bernoulli(0.41) per row,
+      one planted needle per flagged row;
+  mixed: batch 32, one layer, t uniform in [4096, 65536] per row, Full calls
+      Bernoulli(--rate) per row;
+  recall: batch 16, one layer, t = --context (4096 or 131072) for every row,
+      the recall head's own scores decide the gate (theta = 0).
+Every workload runs the 6144 -> 4096 -> 1 recall head each step. One "step"
+= one decode step of the whole path (append, Local per layer, recall head with
+the gate, Full per layer when a row is flagged) replayed from a captured CUDA
+graph; inputs are resident in HBM and fed with one device copy per step.
+Workloads whose per-step reads would fit the 126 MB L2 rotate through
+--copies independently allocated copies of the KV state.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl oda|reference]
+                    [--workload ctx128k|ctx16k|mixed|recall] [--rate R] [--context T]
 
 Prints one JSON line (rank 0). Under torchrun every rank runs an independent
 replica (the path has no cross-request exchange) and the time is the max
@@ -21,9 +31,9 @@ from __future__ import annotations
 
 import argparse
 import hashlib
-import re
 import json
 import os
+import re
 import subprocess
 import sys
 import threading
@@ -39,33 +49,51 @@ METRIC = "decode-attn tokens/s & KV GB/s vs HBM roofline, 128K ctx, 12.5% full c
 UNIT = "tokens/s"
 KV_BYTES_PER_TOKEN_LAYER = 2 * 8 * 128 * 2      # K and V, 8 KV heads, d=128, bf16
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0                        # B200 HBM3e, nominal
+WORKLOADS = ("ctx128k", "ctx16k", "mixed", "recall")
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=1024)
     ap.add_argument("--warmup", type=int, default=8)
     ap.add_argument("--impl", choices=["oda", "reference"], default="oda")
-    ap.add_argument("--layers", type=int, default=28)
+    ap.add_argument("--workload", choices=WORKLOADS, default="ctx128k")
+    ap.add_argument("--layers", type=int, default=28, help="layers of the ctx128k workload")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--cpu-steps", type=int, default=8)
+    ap.add_argument("--cpu-steps", type=int, default=4,
+                    help="decode steps in the oracle's bounded sample (a quarter flagged)")
+    ap.add_argument("--cpu-workers", type=int, default=0,
+                    help="oracle worker processes (0: every core this process may use)")
+    ap.add_argument("--copies", type=int, default=0,
+                    help="independent KV-state copies the steps rotate through "
+                         "(0: 1 for ctx128k, 3 otherwise)")
     ap.add_argument("--launch", choices=["graph", "plain"], default="graph",
                     help="graph: captured step with the IF node; plain: the same kernels "
                          "launched one by one (visible to ncu)")
-    ap.add_argument("--context", type=int, default=131072,
-                    help="context length t at the first step (the headline is 131072)")
-    ap.add_argument("--rate", type=float, default=0.125,
-                    help="Full-call rate: Bernoulli per step (the headline is 0.125)")
+    ap.add_argument("--context", type=int, default=None,
+                    help="context length t at the first step (ctx128k: 131072; recall: "
+                         "131072 or 4096)")
+    ap.add_argument("--rate", type=float, default=None,
+                    help="Full-call rate (ctx128k: Bernoulli per step, default 0.125; mixed: "
+                         "Bernoulli per row, default 0.125)")
     ap.add_argument("--mode", choices=["oda", "full-only", "recall-loss"], default="oda",
                     help="full-only: every step appends and runs Full attention in every "
                          "layer, no Local, recall head or gate (dense decode, for the "
-                         "speedup and the short-context crossover); recall-loss: the recall "
-                         "head's training objective over --positions positions")
+                         "speedup and the short-context crossover; ctx128k only); recall-loss: "
+                         "the recall head's training objective over --positions positions")
     ap.add_argument("--positions", type=int, default=1 << 24,
                     help="positions per recall-loss call (--mode recall-loss)")
-    return ap.parse_args()
+    a = ap.parse_args(argv)
+    if a.context is None:
+        a.context = 131072
+    if a.rate is None and a.workload in ("ctx128k", "mixed"):
+        a.rate = 0.125
+    if a.mode == "full-only" and a.workload != "ctx128k":
+        ap.error("--mode full-only runs the ctx128k request only")
+    return a
 
 
 # ----------------------------------------------------------------------------
@@ -172,13 +200,44 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------
-# algorithmic bytes (KV actually read + KV written)
+# workloads and their algorithmic bytes (KV actually read + KV written)
 # ----------------------------------------------------------------------------
 
+def make_workload(args, n_steps: int):
+    """(Workload, external_scores) for --workload with n_steps decode steps.
+    external_scores: the gate reads the workload's drawn flags (as +-1
+    scores) instead of the recall head's output."""
+    import synth
+    wl = getattr(args, "workload", "ctx128k")
+    rate = getattr(args, "rate", None)
+    if wl == "ctx128k":
+        w = synth.ctx128k(steps=n_steps, layers=getattr(args, "layers", 28),
+                          context=getattr(args, "context", None) or 131072,
+                          rate=0.125 if rate is None else rate)
+    elif wl == "ctx16k":
+        w = synth.ctx16k(steps=n_steps)
+    elif wl == "mixed":
+        w = synth.mixed_batch(0.125 if rate is None else rate, steps=n_steps)
+    elif wl == "recall":
+        w = synth.recall_step(getattr(args, "context", None) or 131072, steps=n_steps)
+        return w, False
+    else:
+        raise ValueError(wl)
+    w.recall = True                  # the recall head runs every step
+    return w, True
+
+
 def step_kv_bytes(t: int, flagged: bool, layers: int, s=4, w=2048) -> int:
+    """One row's algorithmic KV bytes of one step at context t."""
     local = min(t, s + w)
     full = t if flagged else 0
     return layers * (local + full + 2) * KV_BYTES_PER_TOKEN_LAYER
+
+
+def batch_step_bytes(w, j: int, flags_j) -> int:
+    """All rows of step j: Local reads, Full reads of flagged rows, appended K/V."""
+    return sum(step_kv_bytes(int(w.t0[b]) + j, bool(flags_j[b]), w.layers, w.sink, w.window)
+               for b in range(w.batch))
 
 
 def gpu_id(local: int) -> str:
@@ -254,73 +313,177 @@ def recorded_traffic():
 
 # ----------------------------------------------------------------------------
 # the CPU oracle on a bounded sample (cpu_baseline leg and --impl reference)
+#
+# A sample of (kind, row, layer, KV head) tasks of a few decode steps is split
+# over a pool of worker processes (started with spawn, one BLAS thread each).
+# Each worker generates its tasks' inputs first; then all pass a barrier and
+# the parent times the oracle calls alone, from the barrier to the last
+# worker's end. A full step's time is extrapolated from the per-task means
+# and the measured parallel speedup, and every factor is reported.
 # ----------------------------------------------------------------------------
 
-class OracleSample:
-    """Oracle inputs for the sample: Local on layer 0 (all 8 KV heads), Full on
-    layer 0 KV head 0, the recall head for batch row 0. Generating them is not
-    timed; the oracle calls are."""
+def _wl_spec(args) -> dict:
+    return {"workload": getattr(args, "workload", "ctx128k"), "layers": getattr(args, "layers", 28),
+            "context": getattr(args, "context", None), "rate": getattr(args, "rate", None)}
 
-    def __init__(self, w, t_max: int):
-        import oracle as O  # noqa: F401  (test infrastructure; baseline leg only)
-        from synth.gen import table_values
-        self.w = w
-        d, tab = w.d, w.kv_table()
-        lo = max(1, int(w.t0[0]) - w.window)
-        self.Kl, self.Vl = [], []
-        for g in range(w.hkv):
-            K = np.zeros((1, t_max, d))
-            V = np.zeros((1, t_max, d))
-            for kv, dst in ((0, K), (1, V)):
-                key = w.kv_key(0, 0, g, kv)
-                dst[0, :w.sink] = w.to_f64(table_values(key, 0, w.sink * d, tab).reshape(-1, d))
-                dst[0, lo - 1:t_max] = w.to_f64(
-                    table_values(key, (lo - 1) * d, (t_max - lo + 1) * d, tab).reshape(-1, d))
-            self.Kl.append(K)
-            self.Vl.append(V)
-        self.Kf = np.zeros((1, t_max, d))
-        self.Vf = np.zeros((1, t_max, d))
-        self.Kf[0] = w.to_f64(table_values(w.kv_key(0, 0, 0, 0), 0, t_max * d, tab).reshape(-1, d))
-        self.Vf[0] = w.to_f64(table_values(w.kv_key(0, 0, 0, 1), 0, t_max * d, tab).reshape(-1, d))
-        W1, b1, w2, b2 = w.recall_weights()
-        from synth import bf16_bits_to_f32
-        self.W1 = bf16_bits_to_f32(W1).astype(np.float64)
-        self.b1 = b1.astype(np.float64)
-        self.w2 = bf16_bits_to_f32(w2).astype(np.float64)
-        self.b2 = float(b2)
 
-    def step_seconds(self, step: int, flagged: bool) -> float:
-        """Extrapolated seconds for one full decode step (28 layers)."""
-        import oracle as O
+def _kv_rows(w, layer, row, g, positions):
+    """float64 K, V [1][t][d] of one (layer, row, KV head) holding the listed
+    positions (others 0), from the shared seeded generator."""
+    from synth.gen import table_values
+    pos = sorted(positions)
+    t = pos[-1]
+    K = np.zeros((1, t, w.d))
+    V = np.zeros((1, t, w.d))
+    tab = w.kv_table()
+    runs, start, prev = [], pos[0], pos[0]
+    for p in pos[1:]:
+        if p != prev + 1:
+            runs.append((start, prev))
+            start = p
+        prev = p
+    runs.append((start, prev))
+    for kv, dst in ((0, K), (1, V)):
+        key = w.kv_key(layer, row, g, kv)
+        for a, b in runs:
+            vals = table_values(key, (a - 1) * w.d, (b - a + 1) * w.d, tab).reshape(-1, w.d)
+            dst[0, a - 1:b] = w.to_f64(vals)
+        if kv == 0:
+            for n in w.needles:
+                if (n.layer, n.row, n.kv_head) == (layer, row, g) and n.position <= t:
+                    dst[0, n.position - 1] = w.to_f64(n.key)
+    return K, V
+
+
+def _prepare_task(w, task, cache):
+    import oracle as O  # test infrastructure; only the baseline leg runs it
+    kind, j, layer, row, g = task
+    if kind == "recall":
         from synth import bf16_bits_to_f32
-        w = self.w
-        t = int(w.t0[0]) + step
-        q = w.to_f64(w.q_step_layer(step, 0)[0])             # [hq][d] of row 0, layer 0
-        hs = [bf16_bits_to_f32(h).astype(np.float64) for h in w.hidden_step(step)]
-        G = w.group
-        t0 = time.perf_counter()
-        for g in range(w.hkv):
-            O.local_attention(q[g * G:(g + 1) * G], self.Kl[g], self.Vl[g], t, w.sink, w.window)
-        t_local = time.perf_counter() - t0
-        t0 = time.perf_counter()
-        score = O.recall_score(*hs, self.W1, self.b1, self.w2, self.b2)
+        if "W" not in cache:
+            W1, b1, w2, b2 = w.recall_weights()
+            cache["W"] = (bf16_bits_to_f32(W1).astype(np.float64), b1.astype(np.float64),
+                          bf16_bits_to_f32(w2).astype(np.float64), float(b2))
+        hs = [bf16_bits_to_f32(h).astype(np.float64) for h in w.hidden_step(j)]
+        return (kind, hs, cache["W"])
+    t = int(w.t0[row]) + j
+    G = w.group
+    q = w.to_f64(w.q_step_layer(j, layer)[row][g * G:(g + 1) * G])
+    if kind == "local":
+        K, V = _kv_rows(w, layer, row, g, O.local_access_set(t, w.sink, w.window))
+    else:
+        K, V = _kv_rows(w, layer, row, g, range(1, t + 1))
+    return (kind, q, K, V, t)
+
+
+def _run_task(w, prep):
+    import oracle as O
+    if prep[0] == "recall":
+        _, hs, (W1, b1, w2, b2) = prep
+        score = O.recall_score(*hs, W1, b1, w2, b2)
         O.gate(score.astype(np.float32), 0.0)
-        t_recall = time.perf_counter() - t0
-        t_full = 0.0
-        if flagged:
-            t0 = time.perf_counter()
-            O.full_attention(q[0:G], self.Kf, self.Vf, t)
-            t_full = time.perf_counter() - t0
-        return w.layers * t_local + t_recall + w.layers * w.hkv * t_full
+    elif prep[0] == "local":
+        _, q, K, V, t = prep
+        O.local_attention(q, K, V, t, w.sink, w.window)
+    else:
+        _, q, K, V, t = prep
+        O.full_attention(q, K, V, t)
 
 
-def blas_threads() -> int:
+def _oracle_worker(spec, n_steps, tasks, start_barrier, out_q):
+    """One worker process: generate the inputs of its tasks, wait at the
+    barrier, time each oracle call."""
+    import types
+    w, _ = make_workload(types.SimpleNamespace(**spec), n_steps)
+    cache = {}
+    prepared = [(task[0], _prepare_task(w, task, cache)) for task in tasks]
+    start_barrier.wait()
+    res = []
+    for kind, prep in prepared:
+        t0 = time.perf_counter()
+        _run_task(w, prep)
+        res.append((kind, time.perf_counter() - t0))
+    out_q.put(res)
+
+
+def oracle_sample(args, w, flags, timed_records):
+    """The bounded oracle sample on this host's cores; the cpu_baseline dict.
+    flags: [records][B]; timed_records: the record index of every timed step."""
+    import multiprocessing as mp
+    steps = cpu_sample_steps(sorted(set(timed_records)), flags.max(axis=1),
+                             max(1, getattr(args, "cpu_steps", 4)))
+    tasks = []
+    n_rows_l = min(w.batch, 2)
+    for j in steps:
+        for b in range(n_rows_l):
+            for g in range(w.hkv):
+                tasks.append(("local", j, 0, b, g))
+        fl = [b for b in range(w.batch) if flags[j][b]]
+        for b in fl[:1]:
+            for g in range(w.hkv):
+                tasks.append(("full", j, 0, b, g))
+        if w.recall:
+            tasks.append(("recall", j, 0, 0, 0))
+    cores = len(os.sched_getaffinity(0))
+    C = getattr(args, "cpu_workers", 0) or cores
+    C = max(1, min(C, len(tasks)))
+    # heavy tasks first, dealt round robin
+    order = sorted(tasks, key=lambda t: {"full": 0, "recall": 1, "local": 2}[t[0]])
+    per_worker = [order[i::C] for i in range(C)]
+    ctx = mp.get_context("spawn")
+    blas = ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS")
+    old = {k: os.environ.get(k) for k in blas}
+    for k in blas:
+        os.environ[k] = "1"            # inherited by the spawned workers
     try:
-        from threadpoolctl import threadpool_info
-        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
-        return int(max(n)) if n else 1
-    except Exception:
-        return 1
+        bar = ctx.Barrier(C + 1)
+        q = ctx.Queue()
+        procs = [ctx.Process(target=_oracle_worker, args=(_wl_spec(args), w.steps, ts, bar, q))
+                 for ts in per_worker]
+        for p in procs:
+            p.start()
+        bar.wait(timeout=1800)
+        t0 = time.perf_counter()
+        results = [q.get(timeout=1800) for _ in procs]
+        wall = time.perf_counter() - t0
+        for p in procs:
+            p.join(timeout=60)
+    finally:
+        for k, v in old.items():
+            if v is None:
+                os.environ.pop(k, None)
+            else:
+                os.environ[k] = v
+    by = {}
+    for res in results:
+        for kind, sec in res:
+            by.setdefault(kind, []).append(sec)
+    mean = {k: float(np.mean(v)) for k, v in by.items()}
+    task_s = float(sum(sum(v) for v in by.values()))
+    speedup = task_s / wall if wall > 0 else 1.0
+    # tasks of an average timed step
+    nf = float(np.mean([flags[j].sum() for j in timed_records]))
+    per_step = {"local": float(w.batch * w.layers * w.hkv), "full": nf * w.layers * w.hkv,
+                "recall": 1.0 if w.recall else 0.0}
+    full_mean = mean.get("full")
+    if full_mean is None:      # no flagged step sampled: a Local task scaled by length
+        tmean = float(np.mean(w.t0))
+        full_mean = mean.get("local", 0.0) * tmean / min(tmean, w.sink + w.window)
+    cpu_s = (per_step["local"] * mean.get("local", 0.0) + per_step["full"] * full_mean +
+             per_step["recall"] * mean.get("recall", 0.0))
+    step_s = cpu_s / speedup
+    counts = {k: len(v) for k, v in by.items()}
+    text = (f"{w.name}: decode steps {list(map(int, steps))}; float64 oracle tasks {counts} "
+            f"(Local: rows 0..{n_rows_l - 1}, layer 0, every KV head; Full: the first flagged "
+            f"row, layer 0, every KV head; recall head + gate: the batch) on {C} worker "
+            f"processes of one thread; {task_s:.2f} s of oracle calls in {wall:.2f} s wall "
+            f"(inputs generated before the clock); a step = sum over its tasks of the mean "
+            f"task seconds / the measured parallel speedup")
+    return {"value": w.batch / step_s, "unit": UNIT, "cores": C, "kind": "oracle",
+            "sample": text, "extrapolated": True, "sample_wall_s": wall,
+            "sample_task_s": task_s, "parallel_speedup": speedup,
+            "task_s": mean, "tasks_per_step": per_step, "sample_tasks": counts,
+            "seconds_per_step": step_s}
 
 
 def cpu_sample_steps(candidates, flags, n: int):
@@ -331,21 +494,26 @@ def cpu_sample_steps(candidates, flags, n: int):
     return sorted(fl[:nf] + un[:max(1, n - nf)])
 
 
-def weighted_step_seconds(secs: dict, flags, rate: float) -> float:
-    """Mean seconds per step at the realised Full-call rate."""
-    un = [v for i, v in secs.items() if not flags[i]]
-    fl = [v for i, v in secs.items() if flags[i]]
-    t_un = float(np.mean(un)) if un else 0.0
-    t_fl = float(np.mean(fl)) if fl else t_un
-    return (1.0 - rate) * t_un + rate * t_fl
+def workload_flags(w):
+    """[steps][B] uint8 flags drawn by the workload (None for the recall
+    workload, whose flags come from the recall head)."""
+    f = w.flags()
+    return None if f is None else f.astype(np.uint8)
 
 
-def sample_text(steps, flags, rate):
-    return (f"decode steps {list(map(int, steps))} ({int(sum(flags))} flagged) of the 128K "
-            f"workload, batch row 0: Local on layer 0 for all 8 KV heads (x28 layers), Full on "
-            f"layer 0 KV head 0 (x28 layers x 8 heads), recall head and gate once per step; "
-            f"float64 oracle; unflagged and flagged step means weighted by the realised "
-            f"Full-call rate {rate:.4f}")
+def oracle_recall_flags(w, steps):
+    """Flags of the recall workload from the oracle's own scores (reference arm)."""
+    import oracle as O
+    from synth import bf16_bits_to_f32
+    W1, b1, w2, b2 = w.recall_weights()
+    W1 = bf16_bits_to_f32(W1).astype(np.float64)
+    w2 = bf16_bits_to_f32(w2).astype(np.float64)
+    flags = np.zeros((w.steps, w.batch), np.uint8)
+    for j in sorted(set(steps)):
+        hs = [bf16_bits_to_f32(h).astype(np.float64) for h in w.hidden_step(j)]
+        s = O.recall_score(*hs, W1, b1.astype(np.float64), w2, float(b2))
+        flags[j] = O.gate(s.astype(np.float32), 0.0)[0]
+    return flags
 
 
 # ----------------------------------------------------------------------------
@@ -355,53 +523,61 @@ def sample_text(steps, flags, rate):
 def run_reference(args, rank, ws):
     if rank != 0:
         return
-    import synth
-    w = synth.ctx128k(steps=args.warmup + args.steps, layers=args.layers, context=args.context,
-                      rate=args.rate)
-    w.recall = True
-    flags = w.flags()[:, 0]
-    t_max = int(w.t0[0]) + w.steps
-    sample = OracleSample(w, t_max)
-    for i in range(min(args.warmup, 1)):                 # warm caches and BLAS threads
-        sample.step_seconds(i, bool(flags[i]))
-    steps = list(range(args.warmup, args.warmup + args.steps))
-    rate = float(flags[steps].mean())
-    # every timed step is represented by a bounded sample of at most 16 of
-    # them (flagged and unflagged in proportion, at least one flagged when
-    # any is), so the run ends within minutes whatever K is
-    timed_steps = cpu_sample_steps(steps, flags, min(len(steps), 16))
-    secs = {i: sample.step_seconds(i, bool(flags[i])) for i in timed_steps}
-    per_step = weighted_step_seconds(secs, flags, rate)
-    value = w.batch / per_step
-    cores = blas_threads()
+    W, K = args.warmup, args.steps
+    w, external = make_workload(args, W + K)
+    timed = list(range(W, W + K))
+    flags = workload_flags(w)
+    if flags is None:
+        flags = oracle_recall_flags(w, timed)
+    cpu = oracle_sample(args, w, flags, timed)
+    value = cpu["value"]
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
-        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": 1000.0 * per_step, "higher_is_better": True,
+        "n_gpus": getattr(args, "gpus", 1), "steps": K, "warmup": W,
+        "ms_per_step": 1000.0 * cpu["seconds_per_step"], "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": config_block(w, args, ws),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": sample_text(timed_steps, flags[timed_steps], rate)},
+        "cpu_baseline": cpu,
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
 
-def config_block(w, args, ws):
+def config_block(w, args, ws, copies: int = 1):
     mode = getattr(args, "mode", "oda")
-    desc = (f"{w.name}: batch 1, {w.layers} layers, 16/8 heads, d=128, bf16, "
-            f"t={int(w.t0[0])}+step, s=4, w=2048, ")
-    desc += ("Full calls Bernoulli(%g) per step, recall head 6144->4096->1" % w.flag_rate
-             if mode == "oda" else "dense decode: append + Full attention every layer, every step")
-    return {"workload": desc, "mode": mode,
+    wl = getattr(args, "workload", "ctx128k")
+    t0 = [int(x) for x in w.t0]
+    ctx_desc = f"t={t0[0]}+step" if len(set(t0)) == 1 else f"t in [{min(t0)}, {max(t0)}]+step"
+    desc = (f"{w.name}: batch {w.batch}, {w.layers} layers, {w.hq}/{w.hkv} heads, d={w.d}, "
+            f"{w.dtype}, {ctx_desc}, s={w.sink}, w={w.window}, ")
+    if mode == "full-only":
+        desc += "dense decode: append + Full attention every layer, every step"
+        rate = 1.0
+    elif wl == "recall":
+        desc += "recall head 6144->4096->1 scores decide the gate (theta=0)"
+        rate = None
+    else:
+        rate = w.flag_rate
+        per = "step" if w.flag_per == "step" else "row"
+        desc += (f"Full calls Bernoulli({w.flag_rate:g}) per {per}, "
+                 f"recall head 6144->4096->1 every step")
+    local_mb = (w.layers * sum(min(t, w.sink + w.window) for t in t0)
+                * KV_BYTES_PER_TOKEN_LAYER / 1e6)
+    cache_gb = w.layers * sum(t0) * KV_BYTES_PER_TOKEN_LAYER / 1e9
+    if copies > 1:
+        l2 = (f"the steps rotate through {copies} independently allocated copies of the KV "
+              f"state and recall weights (Local reads {local_mb:.0f} MB per step)")
+    else:
+        l2 = ("no flush needed: per-step reads (ring %d MB, Full %d GB) exceed the 126 MB L2"
+              % (round(local_mb), round(cache_gb)))
+    return {"workload": desc, "mode": mode, "name": w.name,
             "batch_per_gpu": int(w.batch), "global_batch": int(w.batch * ws),
-            "context": int(w.t0[0]), "layers": int(w.layers), "hq": w.hq, "hkv": w.hkv,
+            "context": t0[0] if len(set(t0)) == 1 else [min(t0), max(t0)],
+            "layers": int(w.layers), "hq": w.hq, "hkv": w.hkv,
             "head_dim": w.d, "sink": w.sink, "window": w.window,
-            "full_call_rate": w.flag_rate if mode == "oda" else 1.0,
+            "full_call_rate": rate,
             "parallelism": f"replicas x{ws}", "launch": getattr(args, "launch", "graph"),
-            "l2": "no flush needed: per-step reads (ring %d MB, Full %d GB) exceed the 126 MB L2"
-                  % (round(w.layers * min(int(w.t0[0]), w.sink + w.window) * KV_BYTES_PER_TOKEN_LAYER / 1e6),
-                     round(w.layers * int(w.t0[0]) * KV_BYTES_PER_TOKEN_LAYER / 1e9))}
+            "copies": copies, "l2": l2}
 
 
 # ----------------------------------------------------------------------------
@@ -449,82 +625,115 @@ def run_recall_loss(args, rank, ws, local):
             "config": {"workload": f"oda_recall_loss over {n} positions", "positions": n,
                        "l2": "inputs of %d MB exceed the 126 MB L2" % (12 * n // 10**6)},
             "roofline": {"bound": "hbm", "achieved": gbs / ws, "peak": hbm, "unit": "GB/s",
-                         "frac": gbs / ws / hbm, "traffic": None, "peak_kind": kind},
+                         "frac": gbs / ws / hbm, "frac_of_nominal": gbs / ws / NOMINAL_HBM_GBS,
+                         "traffic": None, "peak_kind": kind},
             "device_error": err}), flush=True)
+
+
+def device_flags(ctx, st, recs, r, n_rec, w, torch):
+    """Flags of every record from the recall head's own scores, computed on the
+    device by the same kernels as in the step (untimed)."""
+    scores = torch.empty(w.batch, dtype=torch.float32, device="cuda")
+    fl = torch.empty(w.batch, dtype=torch.uint8, device="cuda")
+    idx = torch.empty(w.batch, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(1, dtype=torch.int32, device="cuda")
+    out = np.zeros((n_rec, w.batch), np.uint8)
+    for j in range(n_rec):
+        ctx.recall_score(st.record_view(recs, j, "h_prev"), st.record_view(recs, j, "emb"),
+                         st.record_view(recs, j, "h_local"), r["H"], r["W1"], r["b1"], r["w2"],
+                         r["b2"], r["hidden"], scores, w.batch)
+        ctx.gate(scores, 0.0, w.batch, fl, idx, cnt)
+        out[j] = fl.cpu().numpy()
+    return out
 
 
 def run_oda(args, rank, ws, local):
     import torch
 
-    import synth
     from gated_local_full_b200 import oda
     from gated_local_full_b200.runtime import DecodeStep
     from synth.device import DeviceWorkload
 
     torch.cuda.set_device(local)
     K, W = args.steps, args.warmup
-    w = synth.ctx128k(steps=W + K, layers=args.layers, context=args.context, rate=args.rate)
-    w.recall = True                                   # recall head runs every step
-    flags = w.flags()[:, 0]
+    S = W + K
+    dense = args.mode == "full-only"
+    R = args.copies or (1 if args.workload == "ctx128k" else 3)
+    n_rec = (S + R - 1) // R                     # step i runs copy i % R on record i // R
+    w, external = make_workload(args, n_rec)
     bt, nb = w.paging()
     cfg = oda.make_config(layers=w.layers, max_batch=w.batch, hq=w.hq, hkv=w.hkv, head_dim=w.d,
                           sink=w.sink, window=w.window, dtype=w.dtype,
                           max_blocks_per_seq=bt.shape[1], num_blocks=nb)
     ctx = oda.OdaContext(cfg)
-    dw = DeviceWorkload(w, ctx.layout, w.batch)
-    pre = torch.from_numpy((w.t0 - 1).astype(np.int32)).cuda()
-    ctx.ring_init(0, w.layers, pre, dw.block_table, dw.cache, dw.ring, w.batch)
-    st = DecodeStep(ctx, w.batch, dw.cache, dw.ring, dw.block_table, recall=dw.recall,
-                    external_scores=True, graph=(args.launch == "graph"))
-    S = W + K
-    recs = st.new_records(S)
-    r = dw.recall
-    for i in range(S):
-        st.pack(recs, i, q=dw.q[i], k_new=dw.k_new[i], v_new=dw.v_new[i],
-                seq_lens=dw.seq_lens[i], gate_scores=dw.scores[i], h_prev=r["h_prev"][i],
-                emb=r["emb"][i], h_local=r["h_local"][i])
-    del dw.q, dw.k_new, dw.v_new
+    copies = []
+    for c in range(R):
+        dw = DeviceWorkload(w, ctx.layout, w.batch)
+        pre = torch.from_numpy((w.t0 - 1).astype(np.int32)).cuda()
+        ctx.ring_init(0, w.layers, pre, dw.block_table, dw.cache, dw.ring, w.batch)
+        st = DecodeStep(ctx, w.batch, dw.cache, dw.ring, dw.block_table, recall=dw.recall,
+                        external_scores=external, graph=(args.launch == "graph"))
+        copies.append((dw, st))
+    dw0, st0 = copies[0]
+    recs = st0.new_records(n_rec)
+    r = dw0.recall
+    for j in range(n_rec):
+        st0.pack(recs, j, q=dw0.q[j], k_new=dw0.k_new[j], v_new=dw0.v_new[j],
+                 seq_lens=dw0.seq_lens[j], gate_scores=dw0.scores[j] if external else None,
+                 h_prev=r["h_prev"][j], emb=r["emb"][j], h_local=r["h_local"][j])
+    for dw, _ in copies:
+        del dw.q, dw.k_new, dw.v_new
     torch.cuda.synchronize()
     assert ctx.get_device_error() == 0
     stream = torch.cuda.current_stream()
+    flags = workload_flags(w) if external else device_flags(ctx, st0, recs, r, n_rec, w, torch)
 
-    dense = args.mode == "full-only"
+    def step_of(i):
+        return copies[i % R], i // R
+
     if dense:
         # dense decode on the same kernels: commit the token, then Full
         # attention for every row in every layer, captured once as a graph
         cnt_all = torch.full((1,), w.batch, dtype=torch.int32, device="cuda")
         idx_all = torch.arange(w.batch, dtype=torch.int32, device="cuda")
+        dgraphs = []
+        for dw, st in copies:
+            def dense_step(dw=dw, st=st):
+                ctx.append_kv(0, w.layers, st.k_new, st.v_new, st.seq_lens, dw.block_table,
+                              dw.cache, dw.ring, w.batch)
+                for l in range(w.layers):
+                    ctx.full_attn_gated(l, st.q[l], st.seq_lens, dw.block_table, dw.cache,
+                                        idx_all, cnt_all, st.out[l], None, w.batch,
+                                        inputs_ready=l > 0)
+            side = torch.cuda.Stream()
+            side.wait_stream(stream)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=side):
+                dense_step()
+            stream.wait_stream(side)
+            dgraphs.append(g)
 
-        def dense_step():
-            ctx.append_kv(0, w.layers, st.k_new, st.v_new, st.seq_lens, dw.block_table, dw.cache,
-                          dw.ring, w.batch)
-            for l in range(w.layers):
-                ctx.full_attn_gated(l, st.q[l], st.seq_lens, dw.block_table, dw.cache, idx_all,
-                                    cnt_all, st.out[l], None, w.batch, inputs_ready=l > 0)
-
-        side = torch.cuda.Stream()
-        side.wait_stream(stream)
-        dgraph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(dgraph, stream=side):
-            dense_step()
-        stream.wait_stream(side)
-        run_step = dgraph.replay
+        def run_step(i):
+            (dw, st), j = step_of(i)
+            st.feed_record(recs, j)
+            dgraphs[i % R].replay()
     else:
-        run_step = st.run
+        def run_step(i):
+            (dw, st), j = step_of(i)
+            st.feed_record(recs, j)
+            st.run()
 
     sampler = ClockSampler(gpu_id(local))
     for i in range(W):
-        st.feed_record(recs, i)
-        run_step()
+        run_step(i)
     torch.cuda.synchronize()
     barrier(ws)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     h0 = time.time()
     e0.record(stream)
-    for i in range(W, W + K):
-        st.feed_record(recs, i)
-        run_step()
+    for i in range(W, S):
+        run_step(i)
     e1.record(stream)
     torch.cuda.synchronize()
     h1 = time.time()
@@ -534,96 +743,142 @@ def run_oda(args, rank, ws, local):
     sampler.stop()              # nvidia-smi no longer competes with the legs below
     err = ctx.get_device_error()
     t_max = max_over_ranks(elapsed, ws)
-    timed = list(range(W, W + K))
-    n_flag = int(flags[timed].sum())
+    timed = list(range(W, S))
+    recs_timed = [i // R for i in timed]
+    n_flag_rows = int(sum(flags[j].sum() for j in recs_timed))
+    n_flag_steps = int(sum(1 for j in recs_timed if flags[j].any()))
     if dense:
-        kv_bytes = sum(w.layers * (int(w.t0[0]) + i + 2) * KV_BYTES_PER_TOKEN_LAYER
-                       for i in timed)
+        kv_bytes = sum(w.layers * sum(int(w.t0[b]) + j + 2 for b in range(w.batch))
+                       * KV_BYTES_PER_TOKEN_LAYER for j in recs_timed)
         launches = K * (w.layers + 1)
     else:
-        kv_bytes = sum(step_kv_bytes(int(w.t0[0]) + i, bool(flags[i]), w.layers) for i in timed)
-        # append, Local x L, recall, gate, then Full x L: behind the IF node
-        # only flagged steps launch them; plain launches issue them every step
-        launches = K * (w.layers + 4) + (n_flag if args.launch == "graph" else K) * w.layers
+        kv_bytes = sum(batch_step_bytes(w, j, flags[j]) for j in recs_timed)
+        # append, Local x L, the recall head (its last CTA gates), then Full x L:
+        # behind the IF node only steps with a flagged row launch them; plain
+        # launches issue the gate and the Full launches every step
+        if args.launch == "graph":
+            launches = K * (w.layers + 2) + n_flag_steps * w.layers
+        else:
+            launches = K * (2 * w.layers + 3)
 
-    # ---- dominant kernel: Full attention. As in a flagged step, the L layers'
-    # launches run back to back: the runs of up to 16 flagged steps are
-    # captured in one CUDA graph (no host launch cost between kernels), which
-    # is replayed between two CUDA events on this stream; the average launch
-    # duration is the replay's time over its launches.
-    cnt1 = torch.ones(1, dtype=torch.int32, device="cuda")
-    idx0 = torch.zeros(w.batch, dtype=torch.int32, device="cuda")
-    outb = torch.empty_like(st.out[0])
-    fl_steps = [i for i in timed if flags[i]][:16] or [timed[0]]
+    # ---- per-kernel launch times, as in a step: the L layers' launches back
+    # to back (flag set from the second on), for up to 16 timed steps, each on
+    # its own copy, captured in one CUDA graph and replayed between two CUDA
+    # events on this stream
+    outb = torch.empty_like(st0.out[0])
+    ids = {}
+    for j in sorted(set(recs_timed)):
+        rows = [b for b in range(w.batch) if flags[j][b]]
+        if rows:
+            idx = torch.full((w.batch,), -1, dtype=torch.int32)
+            idx[:len(rows)] = torch.tensor(rows, dtype=torch.int32)
+            ids[j] = (idx.cuda(), torch.tensor([len(rows)], dtype=torch.int32, device="cuda"))
+    fl_steps = [i for i in timed if (i // R) in ids][:16]
+    loc_steps = timed[:16]
 
     def run_full():
         for i in fl_steps:
-            q = st.record_view(recs, i, "q")
-            sl = st.record_view(recs, i, "seq_lens")
+            (dw, st), j = step_of(i)
+            q = st.record_view(recs, j, "q")
+            sl = st.record_view(recs, j, "seq_lens")
+            idx, cnt = ids[j]
             for l in range(w.layers):
-                ctx.full_attn_gated(l, q[l], sl, dw.block_table, dw.cache, idx0, cnt1, outb,
-                                    None, w.batch, inputs_ready=l > 0)
+                ctx.full_attn_gated(l, q[l], sl, dw.block_table, dw.cache, idx, cnt, outb, None,
+                                    w.batch, inputs_ready=l > 0)
 
     def run_local():
-        for i in timed[:16]:
-            q = st.record_view(recs, i, "q")
-            sl = st.record_view(recs, i, "seq_lens")
+        for i in loc_steps:
+            (dw, st), j = step_of(i)
+            q = st.record_view(recs, j, "q")
+            sl = st.record_view(recs, j, "seq_lens")
             for l in range(w.layers):
                 ctx.local_attn(l, q[l], sl, dw.ring, outb, None, w.batch, inputs_ready=l > 0)
 
-    full_s, n_full = replay_seconds(torch, run_full, stream), len(fl_steps) * w.layers
-    local_s, n_local = replay_seconds(torch, run_local, stream), min(K, 16) * w.layers
-    full_bytes = sum((int(w.t0[0]) + i) * KV_BYTES_PER_TOKEN_LAYER for i in fl_steps) * w.layers
-    full_gbs = float(full_bytes / full_s / 1e9)
-    local_us = float(local_s / n_local * 1e6)
     hbm, hbm_kind = peaks()
-    traffic, _ = recorded_traffic()
+    kernels = {}
+    local_s = replay_seconds(torch, run_local, stream)
+    n_local = len(loc_steps) * w.layers
+    local_bytes = sum(sum(min(int(w.t0[b]) + i // R, w.sink + w.window) for b in range(w.batch))
+                      for i in loc_steps) * w.layers * KV_BYTES_PER_TOKEN_LAYER
+    kernels["local"] = {"kernel": "attn_kernel<bf16,128,2,RING=true> (Local attention)",
+                        "mean_launch_us": local_s / n_local * 1e6,
+                        "bytes_per_launch": local_bytes / n_local,
+                        "achieved_gbs": local_bytes / local_s / 1e9,
+                        "launches_timed": n_local}
+    if fl_steps:
+        full_s = replay_seconds(torch, run_full, stream)
+        n_full = len(fl_steps) * w.layers
+        full_bytes = sum(sum(int(w.t0[b]) + i // R for b in range(w.batch) if flags[i // R][b])
+                         for i in fl_steps) * w.layers * KV_BYTES_PER_TOKEN_LAYER
+        kernels["full"] = {"kernel": "attn_kernel<bf16,128,2,RING=false> (Full attention)",
+                           "mean_launch_us": full_s / n_full * 1e6,
+                           "bytes_per_launch": full_bytes / n_full,
+                           "achieved_gbs": full_bytes / full_s / 1e9,
+                           "launches_timed": n_full}
+    for k in kernels.values():
+        k["frac_of_peak"] = k["achieved_gbs"] / hbm
+        k["frac_of_nominal"] = k["achieved_gbs"] / NOMINAL_HBM_GBS
+    # the dominant kernel: the larger share of an average step's time
+    share_local = kernels["local"]["mean_launch_us"] * w.layers
+    share_full = (kernels["full"]["mean_launch_us"] * w.layers * n_flag_steps / K
+                  if "full" in kernels else 0.0)
+    dom = "full" if share_full >= share_local else "local"
+    traffic = None
+    if dom == "full" and args.workload == "ctx128k":
+        traffic, _ = recorded_traffic()
+    dk = kernels[dom]
+    roofline = {"bound": "hbm", "achieved": dk["achieved_gbs"], "peak": hbm, "unit": "GB/s",
+                "frac": dk["achieved_gbs"] / hbm,
+                "frac_of_nominal": dk["achieved_gbs"] / NOMINAL_HBM_GBS,
+                "traffic": traffic, "kernel": dk["kernel"], "peak_kind": hbm_kind,
+                "launches_timed": dk["launches_timed"],
+                "timing": "CUDA events on the launching stream around a graph replay of L "
+                          "back-to-back launches per step",
+                "mean_launch_us": dk["mean_launch_us"]}
 
     # ---- end to end: host records in, result out, every step
     e2e = None
     if not args.no_e2e:
         # the same K steps as the device-timed run (same Full calls), fed from
         # pinned host memory one step at a time
-        n_e2e = K
-        hrec = st.new_records(n_e2e, pin=True)
-        hrec.copy_(recs[W:W + n_e2e].cpu())
+        hrec = st0.new_records(n_rec, pin=True)
+        hrec.copy_(recs.cpu())
         res = torch.empty((w.batch, w.hq, w.d), dtype=torch.bfloat16).pin_memory()
         cnt = torch.empty(1, dtype=torch.int32).pin_memory()
-        hres = st.new_result()
-        one_call = st.graph is not None and not dense
-        # replays steps W.. on a cache that already holds later positions: the
+        hres = st0.new_result()
+        one_call = st0.graph is not None and not dense
+        # replays steps W.. on caches that already hold later positions: the
         # same work per step; outputs are not checked here
         torch.cuda.synchronize()
         barrier(ws)
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        for j in range(n_e2e):
+        for i in timed:
+            (dw, st), j = step_of(i)
             if one_call:
                 # record in, step graph, last layer's output and count out, wait
                 st.run_io(hrec[j], hres)
             else:
                 st.feed_record(hrec, j)
-                run_step()
+                if dense:
+                    dgraphs[i % R].replay()
+                else:
+                    st.run()
                 res.copy_(st.out[w.layers - 1], non_blocking=True)
                 cnt.copy_(st.count, non_blocking=True)
                 stream.synchronize()
         b.record(stream)
         torch.cuda.synchronize()
         e2e_t = max_over_ranks(a.elapsed_time(b) / 1000.0, ws)
-        e2e = {"value": job_throughput(n_e2e * w.batch, ws, e2e_t), "unit": UNIT,
-               "h2d_bytes_per_step": int(st.record_bytes),
+        e2e = {"value": job_throughput(K * w.batch, ws, e2e_t), "unit": UNIT,
+               "h2d_bytes_per_step": int(st0.record_bytes),
                "d2h_bytes_per_step": int(res.numel() * res.element_size() + 4),
-               "steps": n_e2e}
+               "steps": K, "read_back": "the last layer's output and the flagged-row count"}
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline and not dense:
-        steps = cpu_sample_steps(timed, flags, args.cpu_steps)
-        sample = OracleSample(w, int(w.t0[0]) + S)
-        secs = {i: sample.step_seconds(i, bool(flags[i])) for i in steps}
-        per_step = weighted_step_seconds(secs, flags, n_flag / K)
-        cpu = {"value": w.batch / per_step, "unit": UNIT, "cores": blas_threads(),
-               "kind": "oracle", "sample": sample_text(steps, flags[steps], n_flag / K)}
+        cpu = oracle_sample(args, w, flags, recs_timed)
 
     if rank == 0:
         value = job_throughput(K * w.batch, ws, t_max)
@@ -633,25 +888,21 @@ def run_oda(args, rank, ws, local):
             "warmup": W, "ms_per_step": 1000.0 * t_max / K, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded counter-based generator; no datasets or weights)",
-            "config": config_block(w, args, ws),
+            "config": config_block(w, args, ws, R),
             "kv_gbs": kv_gbs, "kv_frac_of_hbm": kv_gbs / hbm,
+            "kv_frac_of_nominal": kv_gbs / NOMINAL_HBM_GBS,
             "kv_bytes_per_step": kv_bytes / K,
-            "full_call_rate_realised": 1.0 if dense else n_flag / K,
+            "full_call_rate_realised": 1.0 if dense else n_flag_rows / (K * w.batch),
+            "full_steps_realised": n_flag_steps,
             "recall_weight_bytes_per_step": int(w.recall_hidden * 3 * w.hidden * 2),
-            "roofline": {"bound": "hbm", "achieved": full_gbs, "peak": hbm, "unit": "GB/s",
-                         "frac": full_gbs / hbm, "traffic": traffic,
-                         "kernel": "attn_kernel<bf16,128,2,RING=false> (Full attention)",
-                         "peak_kind": hbm_kind,
-                         "launches_timed": n_full,
-                         "timing": "CUDA events on the launching stream around a graph "
-                                   "replay of L back-to-back launches per flagged step",
-                         "mean_launch_us": float(full_s / n_full * 1e6)},
-            "local_attn_mean_launch_us": local_us,
+            "roofline": roofline, "kernels": kernels,
+            "local_attn_mean_launch_us": kernels["local"]["mean_launch_us"],
             "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks, "gpu_launches": launches,
             "device_error": err,
         }
         print(json.dumps(line), flush=True)
-    st.close()
+    for _, st in copies:
+        st.close()
     ctx.close()
 
 

@@ -69,3 +69,37 @@ def test_reference_arm_prints_one_oracle_line():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
+
+
+@pytest.mark.parametrize("wl,extra,name,B", [
+    ("ctx16k", (), "ctx16k_b8", 8),
+    ("mixed", ("--rate", "0.41"), "mixed_b32_rho0.41", 32),
+    ("recall", ("--context", "4096"), "recall_b16_ctx4096", 16),
+])
+def test_other_workloads_and_their_bytes(wl, extra, name, B):
+    """The 16K, mixed-batch and recall-head workloads: shapes, whose scores
+    gate, the L2 rotation note, and the per-step algorithmic bytes (Local
+    min(t, s+w) positions, Full t positions for a flagged row, two appended
+    positions, 4096 bytes per position and layer)."""
+    import bench
+    a = _args("--workload", wl, *extra)
+    w, external = bench.make_workload(a, 3)
+    assert w.name == name and w.batch == B and w.layers == 1 and w.recall
+    assert external == (wl != "recall")
+    c = bench.config_block(w, a, 1, 3)
+    assert c["copies"] == 3 and "3 independently allocated copies" in c["l2"]
+    flags = bench.workload_flags(w)
+    if external:
+        assert flags.shape == (3, B)
+        j = 2
+        want = sum((min(int(w.t0[b]) + j, 2052) + (int(w.t0[b]) + j) * int(flags[j][b]) + 2)
+                   * 4096 for b in range(B))
+        assert bench.batch_step_bytes(w, j, flags[j]) == want
+    else:
+        assert flags is None
+    assert a.mode == "oda" and a.copies == 0
+
+
+def test_full_only_needs_the_headline_request():
+    with pytest.raises(SystemExit):
+        _args("--workload", "mixed", "--mode", "full-only")
