@@ -234,6 +234,15 @@ def step_kv_bytes(t: int, flagged: bool, layers: int, s=4, w=2048) -> int:
     return layers * (local + full + 2) * KV_BYTES_PER_TOKEN_LAYER
 
 
+def model_speedup(t: int, rho: float, s=4, w=2048) -> float:
+    """Dense decode's KV bytes per step over ODA's at Full-call rate rho (both
+    append the token; ODA reads the Local set every step and the whole
+    history on a fraction rho of steps). It tends to 1/rho as t grows."""
+    dense = t + 2
+    oda = min(t, s + w) + rho * t + 2
+    return dense / oda
+
+
 def batch_step_bytes(w, j: int, flags_j) -> int:
     """All rows of step j: Local reads, Full reads of flagged rows, appended K/V."""
     return sum(step_kv_bytes(int(w.t0[b]) + j, bool(flags_j[b]), w.layers, w.sink, w.window)
@@ -904,6 +913,7 @@ def run_oda(args, rank, ws, local):
     for _, st in copies:
         st.close()
     ctx.close()
+    return line if rank == 0 else None
 
 
 def main():

@@ -258,6 +258,25 @@ oda_status oda_full_attn_gated(oda_ctx* ctx, int layer, const void* q, const int
                                (flags & ODA_ATTN_INPUTS_READY) != 0);
 }
 
+oda_status oda_range_attn(oda_ctx* ctx, int layer, const void* q, const int32_t* seq_lens,
+                          const int32_t* range_lo, const int32_t* range_hi,
+                          const int32_t* block_table, const void* kv_cache, const int32_t* idx,
+                          const int32_t* count, void* out, float* lse, int B, unsigned flags,
+                          oda_stream stream) {
+  if (!ctx) return ODA_ERR_ARG;
+  oda_status s = check_batch(ctx, B);
+  if (s != ODA_OK) return s;
+  if (layer < 0 || layer >= ctx->cfg.layers) return ODA_ERR_ARG;
+  if (flags & ~ODA_ATTN_INPUTS_READY) return ODA_ERR_ARG;
+  if (B == 0) return ODA_OK;
+  if (!q || !seq_lens || !range_lo || !range_hi || !block_table || !kv_cache || !idx || !count ||
+      !out)
+    return ODA_ERR_ARG;
+  return oda_impl::launch_attn(ctx, false, layer, q, seq_lens, kv_cache, block_table, idx, count,
+                               out, lse, B, static_cast<cudaStream_t>(stream), nullptr,
+                               (flags & ODA_ATTN_INPUTS_READY) != 0, range_lo, range_hi);
+}
+
 oda_status oda_recall_score(oda_ctx* ctx, const void* h_prev, const void* emb,
                             const void* h_local, int H, const void* W1, const float* b1,
                             const float* w2, float b2, int hidden, float* scores, int B,

@@ -93,6 +93,8 @@ struct AttnArgs {
   const int* plan;              // precomputed partition, or null: compute it here
   int cluster;                  // cluster mode: CTAs per segment (= cluster size)
   int early;                    // stage the first tiles before the dependency wait
+  const int32_t* range_lo;      // paged source: per-row region [lo, hi), or null (1..t)
+  const int32_t* range_hi;
   int* err;
 };
 
@@ -223,6 +225,7 @@ attn_kernel(const AttnArgs a) {
   constexpr int QCH = G * D * (int)sizeof(T) / 16;  // 16-byte chunks of one segment's queries
   uint4* sq = reinterpret_cast<uint4*>(rml + 32 * G);   // [QCH] the current segment's queries
   int* st_t = reinterpret_cast<int*>(sq + QCH);         // cluster mode: the row's t
+  int* rowlo = st_t + 4;                                // paged: [max_batch] first position read
 
   const int tid = threadIdx.x;
   const int lane = tid & 31;
@@ -296,7 +299,9 @@ attn_kernel(const AttnArgs a) {
       pin.grid = (int)gridDim.x;
       pin.err = a.err;
       pin.report = report && blockIdx.x == 0;
-      const PlanHead h = plan_rows(pin, rowb, rowt, rowstart, rowcs);
+      pin.range_lo = a.range_lo;
+      pin.range_hi = a.range_hi;
+      const PlanHead h = plan_rows(pin, rowb, rowt, rowstart, rowcs, RING ? nullptr : rowlo);
       if (lane == 0) {
         int o[5];
         plan_cta((int)blockIdx.x, h, rowstart, rowcs, a.hkv, o);
@@ -342,8 +347,9 @@ attn_kernel(const AttnArgs a) {
             if (ok && jt < a.ring_blocks)
               bulk_prefetch_l2(kb + (((long long)b * a.hkv + ck.g) * a.ring_blocks + jt) * TILE_ELEMS,
                                TILE_BYTES);
-          } else if (ok && jt < a.max_blocks) {
-            const int blk = __ldcg(a.block_table + (long long)b * a.max_blocks + jt);
+          } else if (ok && jt + (rowlo[ck.i] - 1) / ODA_TILE < a.max_blocks) {
+            const int blk = __ldcg(a.block_table + (long long)b * a.max_blocks + jt +
+                                   (rowlo[ck.i] - 1) / ODA_TILE);
             if (blk >= 0 && (long long)blk < a.num_blocks)
               bulk_prefetch_l2(kb + ((long long)blk * a.hkv + ck.g) * TILE_ELEMS, TILE_BYTES);
           }
@@ -447,7 +453,11 @@ attn_kernel(const AttnArgs a) {
   int q0 = 0, q1 = 0, qb0 = -1, qb1 = -1;    // lane 0: grabbed pool tiles, blocks
   auto grab = [&](int& q, int& qb) {         // lane 0 only, after the dependency wait
     q = pool0 + atomicAdd(&a.dyn[sigma0], 1);
-    qb = (!RING && q < seg_nt) ? a.block_table[(long long)seg_b * a.max_blocks + q] : -1;
+    // (the pool belongs to the first segment, row sigma0 / hkv)
+    qb = (!RING && q < seg_nt)
+             ? a.block_table[(long long)seg_b * a.max_blocks +
+                             (rowlo[sigma0 / a.hkv] - 1) / ODA_TILE + q]
+             : -1;
   };
 
   // Block ids of the producer's next 32 tiles of the current row, one per
@@ -491,7 +501,8 @@ attn_kernel(const AttnArgs a) {
           bc_row = i;
           bc_base = jt;
           const int jl = jt + lane * W;
-          bc_val = jl < nt ? a.block_table[(long long)b * a.max_blocks + jl] : -1;
+          const int tb = (rowlo[i] - 1) / ODA_TILE;
+          bc_val = jl < nt ? a.block_table[(long long)b * a.max_blocks + tb + jl] : -1;
         }
         blk = __shfl_sync(0xffffffffu, bc_val, (jt - bc_base) / W);
       }
@@ -619,6 +630,15 @@ attn_kernel(const AttnArgs a) {
     } else {
       t = rowt[seg.i];
     }
+    // paged source: positions first..t are read; relative to the segment's
+    // first tile they are the slots [plo, phi)
+    int plo = 0, phi = t;
+    if constexpr (!RING) {
+      const int first = rowlo[seg.i];
+      const int base = (first - 1) / ODA_TILE * ODA_TILE;
+      plo = first - 1 - base;
+      phi = t - base;
+    }
     const int s0 = seg.s1 - seg.nt;
 
     // this lane's DPL dims of the G query heads (exact, unscaled)
@@ -672,8 +692,7 @@ attn_kernel(const AttnArgs a) {
         const int base = jt * ODA_TILE;
         mask = range_bits(a.sink, a.sink + mw, base) | range_bits(0, nsv, base);
       } else {
-        const int nvalid = min(ODA_TILE, t - jt * ODA_TILE);
-        mask = nvalid >= 16 ? 0xFFFFu : ((1u << nvalid) - 1u);
+        mask = range_bits(plo, phi, jt * ODA_TILE);
       }
       if (badst[warp * NS + stage] || aborted) mask = 0;
 
@@ -1150,6 +1169,7 @@ size_t smem_bytes_wn(int max_batch) {
   s += (size_t)W * NS;
   s += 16 + (size_t)(G * D + 32 * G) * 4;     // cluster mode: pushed accumulators, (m, l)
   s += (size_t)G * D * sizeof(T) + 16;          // the segment's queries, t
+  s += (size_t)max_batch * 4;                   // first position read per row (paged)
   return (s + 127) & ~(size_t)127;
 }
 
@@ -1334,7 +1354,8 @@ oda_status attn_setup(oda_ctx* ctx) {
 oda_status launch_attn(oda_ctx* ctx, bool ring_mode, int layer, const void* q,
                        const int32_t* seq_lens, const void* kv, const int32_t* block_table,
                        const int32_t* idx, const int32_t* count, void* out, float* lse, int B,
-                       cudaStream_t st, const int* plan, bool early) {
+                       cudaStream_t st, const int* plan, bool early, const int32_t* range_lo,
+                       const int32_t* range_hi) {
   const oda_config& c = ctx->cfg;
   AttnArgs a;
   a.q = q;
@@ -1363,6 +1384,8 @@ oda_status launch_attn(oda_ctx* ctx, bool ring_mode, int layer, const void* q,
   a.plan = plan;
   a.cluster = 0;
   a.early = early ? 1 : 0;
+  a.range_lo = ring_mode ? nullptr : range_lo;
+  a.range_hi = ring_mode ? nullptr : range_hi;
   a.err = ctx->err;
   if (ring_mode) return dispatch<true>(c, Launch{ctx, &a, st, true});
   return dispatch<false>(c, Launch{ctx, &a, st, false});
@@ -1529,6 +1552,8 @@ extern "C" oda_status oda_full_attn_gated_static(const oda_config* cfg, int laye
   a.plan = nullptr;
   a.cluster = 0;
   a.early = 0;
+  a.range_lo = nullptr;
+  a.range_hi = nullptr;
   a.err = err ? err : sd->err;
   return dispatch<false>(*cfg, LaunchStatic{&a, sd->num_sms, cfg->max_batch, B, st});
 }

@@ -206,6 +206,8 @@ oda_status launch_append(oda_ctx* ctx, int lb, int le, const void* k_new, const 
     a.pin.grid = ctx->attn_ctas_local;
     a.pin.err = ctx->err;
     a.pin.report = true;
+    a.pin.range_lo = nullptr;
+    a.pin.range_hi = nullptr;
     smem = (size_t)(4 * c.max_batch + 2) * sizeof(int);
   }
   const int grid = a.nblk_append + (local_plan ? 1 : 0);

@@ -236,7 +236,8 @@ oda_status launch_ring_init(oda_ctx* ctx, int lb, int le, const int32_t* seq_len
 oda_status launch_attn(oda_ctx* ctx, bool ring_mode, int layer, const void* q,
                        const int32_t* seq_lens, const void* kv, const int32_t* block_table,
                        const int32_t* idx, const int32_t* count, void* out, float* lse, int B,
-                       cudaStream_t st, const int* plan = nullptr, bool early = false);
+                       cudaStream_t st, const int* plan = nullptr, bool early = false,
+                       const int32_t* range_lo = nullptr, const int32_t* range_hi = nullptr);
 int attn_min_tiles(oda_ctx* ctx, bool ring_mode);
 oda_status attn_setup(oda_ctx* ctx);
 oda_status launch_gate(oda_ctx* ctx, const float* scores, float theta, int B, uint8_t* flags,

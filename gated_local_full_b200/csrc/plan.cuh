@@ -33,15 +33,18 @@ struct PlanIn {
   int grid;                    // CTAs of the attention launch
   int* err;
   bool report;                 // record errors (one block per launch does)
+  const int32_t* range_lo;     // paged source only: per row, first position of the region
+  const int32_t* range_hi;     // ... and one past its last (null: the whole history 1..t)
 };
 
 struct PlanHead {
   int nr, tot, P, al;
 };
 
-// Warp 0 only. Writes rowb/rowt [nr], rowstart/rowcs [nr+1].
+// Warp 0 only. Writes rowb/rowt [nr], rowstart/rowcs [nr+1], and for the
+// paged source rowlo [nr] (the region's first position; rowt is its last).
 __device__ __forceinline__ PlanHead plan_rows(const PlanIn& p, int* rowb, int* rowt,
-                                              int* rowstart, int* rowcs) {
+                                              int* rowstart, int* rowcs, int* rowlo = nullptr) {
   const int lane = threadIdx.x & 31;
   const bool ring = p.count == nullptr;
   // with B <= 32 every lane loads one row's length and one compacted id
@@ -68,19 +71,29 @@ __device__ __forceinline__ PlanHead plan_rows(const PlanIn& p, int* rowb, int* r
     const int ts = __shfl_sync(0xffffffffu, tl, okl ? (bl & 31) : 0);   // all lanes shuffle
     if (i < nr) {
       const int t = !okl ? 0 : (small ? ts : __ldcg(p.seq_lens + bl));
+      int first = 1, last = t;                   // positions first..last are read
       if (!okl || t < 1) {
         if (p.report) record_error(p.err, ODA_ERR_BOUNDS);
       } else if (ring) {
         nt = (p.sink + min(t, p.window) + ODA_TILE - 1) / ODA_TILE;
       } else {
-        nt = (t + ODA_TILE - 1) / ODA_TILE;
-        if (nt > p.max_blocks) {
+        bool ok = true;
+        if (p.range_lo) {                        // the region [lo, hi), within 1..t
+          const int rl = __ldcg(p.range_lo + bl), rh = __ldcg(p.range_hi + bl);
+          ok = rl >= 1 && rh > rl && rh - 1 <= t;
+          first = rl;
+          last = rh - 1;
+        }
+        const int tend = (last + ODA_TILE - 1) / ODA_TILE;   // tiles up to the last position
+        if (!ok || tend > p.max_blocks) {
           if (p.report) record_error(p.err, ODA_ERR_BOUNDS);
-          nt = 0;
+        } else {
+          nt = tend - (first - 1) / ODA_TILE;
         }
       }
       rowb[i] = okl ? bl : 0;
-      rowt[i] = t;
+      rowt[i] = ring ? t : last;
+      if (rowlo) rowlo[i] = first;
     }
     int v = nt * p.hkv;
 #pragma unroll

@@ -33,7 +33,7 @@ EXPORTS = (
     "oda_get_device_error", "oda_selftest_wait_timeout", "oda_step_run",
     "oda_step_graph_create", "oda_step_graph_launch", "oda_step_graph_run_io",
     "oda_step_graph_destroy", "oda_version",
-    "oda_full_attn_gated_static",
+    "oda_full_attn_gated_static", "oda_range_attn",
 )
 
 
@@ -100,6 +100,8 @@ def lib() -> ctypes.CDLL:
         "oda_step_graph_destroy": [vp],
         "oda_full_attn_gated_static": [POINTER(OdaConfig), c_int, vp, vp, vp, vp, vp, vp, vp,
                                        vp, c_int, vp, vp],
+        "oda_range_attn": [vp, c_int, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, c_int,
+                           ctypes.c_uint, vp],
     }
     for name, args in sig.items():
         f = getattr(L, name)
@@ -267,6 +269,16 @@ class OdaContext:
                                          ptr(out), ptr(lse), B,
                                          ATTN_INPUTS_READY if inputs_ready else 0,
                                          _stream(stream)), "oda_full_attn_gated")
+
+    def range_attn(self, layer, q, seq_lens, range_lo, range_hi, block_table, kv_cache, idx,
+                   count, out, lse, B, stream=None, inputs_ready=False):
+        """Attention of the rows idx[0..count) over positions [lo, hi) only
+        (oda_range_attn)."""
+        _check(lib().oda_range_attn(self.handle, layer, ptr(q), ptr(seq_lens), ptr(range_lo),
+                                    ptr(range_hi), ptr(block_table), ptr(kv_cache), ptr(idx),
+                                    ptr(count), ptr(out), ptr(lse), B,
+                                    ATTN_INPUTS_READY if inputs_ready else 0, _stream(stream)),
+               "oda_range_attn")
 
     def get_device_error(self, stream=None) -> int:
         e = c_int(0)

@@ -254,6 +254,27 @@ oda_status oda_full_attn_gated(oda_ctx* ctx, int layer, const void* q,
                                unsigned flags, oda_stream stream);
 
 /*
+ * Range-restricted ("focus") attention: for the rows idx[0..*count), softmax
+ * attention over the positions of one region [lo, hi) of the paged history
+ * only, reading only that region's K/V. The Declarative Attention pages
+ * describe this mode ("<focus>: narrowed to a specific region, reading only
+ * that region's KV cache", zhichai.net post, section "Three Attention
+ * Modes"; kongchang.com article, section "<focus> Mode: Precise Region
+ * Targeting"). For row b with t = seq_lens[b]:
+ *   out[b][h] = sum_{j = lo..hi-1} softmax_j(q[b][h] . k_j / sqrt(d)) v_j,
+ *   lo = range_lo[b], hi = range_hi[b],  1 <= lo < hi <= t + 1
+ * (hi = t + 1 includes the current token; lo = 1, hi = t + 1 is Full).
+ * A region outside those bounds records ODA_ERR_BOUNDS and the row is left
+ * as `out` holds it. Arguments, layouts and flags as for oda_full_attn_gated;
+ * range_lo, range_hi: device int32 [B], indexed by row id like seq_lens.
+ */
+oda_status oda_range_attn(oda_ctx* ctx, int layer, const void* q, const int32_t* seq_lens,
+                          const int32_t* range_lo, const int32_t* range_hi,
+                          const int32_t* block_table, const void* kv_cache, const int32_t* idx,
+                          const int32_t* count, void* out, float* lse, int B, unsigned flags,
+                          oda_stream stream);
+
+/*
  * Full attention for callers that cannot allocate device memory (the pages
  * have no counterpart; this is an interface for integrators). Engines that
  * hand the whole GPU to their own pool allocator at start-up cannot have a

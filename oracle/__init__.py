@@ -10,6 +10,9 @@ Sources (the web pages this oracle restates):
   [CARD] "On-Demand Attention: Language Models Know When to Recall", dair.ai paper card
   [EXPL] "Let models trigger full attention only when recall helps -- On-Demand
          Attention recall-head gating", learnaivisually explainer
+  [DA-1] zhichai.net post on Declarative Attention (the "<focus>" mode)
+  [DA-2] "Declarative Attention: Letting LLMs Control Their Own Attention",
+         kongchang.com article ("<focus> Mode: Precise Region Targeting")
 
 Parity status per function is listed in ``oracle/oda_oracle.py``'s header.
 """

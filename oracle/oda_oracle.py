@@ -16,6 +16,7 @@ Parity status
   access_gain, penalized_step_loss ..... pinned (closed forms)
   delta_F and the FLOP counter ......... pinned (exact integer identity; pages' ratios, loose)
   gelu_erf ............................. pinned (erf closed-form values)
+  range_access_set, range_attention .... pinned (brute force, Full/window/one-position cases)
   recall_score ......................... parity unpinned: the pages give the
       head's inputs and parameter count but not its architecture; the
       6144 -> 4096 -> 1 GELU MLP is this library's stated choice. Pinned only
@@ -37,6 +38,7 @@ __all__ = [
     "recall_regression_loss", "access_gain", "penalized_step_loss",
     "best_action", "regression_target", "attention_flops", "recall_flops",
     "delta_F", "model_step_flops", "oda_flop_fraction",
+    "range_access_set", "range_attention",
 ]
 
 
@@ -127,6 +129,26 @@ def full_attention(q, K, V, t: int, flops: Optional[FlopCounter] = None):
     """F: attention over S^F_t, run only for requests the gate flags
     ([SUM] Methodology / Local-First Decoding)."""
     return attend(q, K, V, full_access_set(t), flops, "full")
+
+
+# ---------------------------------------------------------------------------
+# Range-restricted ("focus") attention. [DA-1] (zhichai.net post on
+# Declarative Attention), "Three Attention Modes", and [DA-2] (kongchang.com
+# article), "<focus> Mode: Precise Region Targeting": attention narrowed to one
+# region of the context, reading only that region's KV. Reading used (the
+# pages give no formula): the region is the half-open position range
+# [lo, hi) named by the caller, and the attention is the same softmax
+# attention restricted to it.
+# ---------------------------------------------------------------------------
+
+def range_access_set(lo: int, hi: int) -> set:
+    """{lo, ..., hi-1}."""
+    return set(range(lo, hi))
+
+
+def range_attention(q, K, V, lo: int, hi: int, flops: Optional[FlopCounter] = None):
+    """Attention over the positions of [lo, hi) only."""
+    return attend(q, K, V, range_access_set(lo, hi), flops, "range")
 
 
 # ---------------------------------------------------------------------------

@@ -138,3 +138,25 @@ def oracle_heads(w: Workload, tasks, workers=None):
         return [_head_task(a) for a in args]
     with cf.ProcessPoolExecutor(max_workers=n, mp_context=mp.get_context("spawn")) as ex:
         return list(ex.map(_head_task, args, chunksize=1))
+
+
+def _range_task(args):
+    w, q_row, layer, row, g, lo, hi = args
+    G = w.group
+    q = w.to_f64(q_row[g * G:(g + 1) * G])
+    K, V = oracle_kv_head(w, layer, row, g, hi - 1, range(lo, hi))
+    return O.range_attention(q, K, V, lo, hi)
+
+
+def oracle_range_heads(w: Workload, tasks, workers=None):
+    """Oracle outputs of range-restricted attention for (q_row, layer, row,
+    kv_head, lo, hi) tasks, in order (a spawn process pool, as oracle_heads)."""
+    import concurrent.futures as cf
+    import multiprocessing as mp
+    import os
+    args = [(w, *t) for t in tasks]
+    n = workers or min(len(os.sched_getaffinity(0)), 16)
+    if len(args) <= 2 or n <= 1:
+        return [_range_task(a) for a in args]
+    with cf.ProcessPoolExecutor(max_workers=n, mp_context=mp.get_context("spawn")) as ex:
+        return list(ex.map(_range_task, args, chunksize=1))

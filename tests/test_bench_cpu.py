@@ -103,3 +103,19 @@ def test_other_workloads_and_their_bytes(wl, extra, name, B):
 def test_full_only_needs_the_headline_request():
     with pytest.raises(SystemExit):
         _args("--workload", "mixed", "--mode", "full-only")
+
+
+def test_bytes_model_speedup_tends_to_inverse_rate():
+    """The pages' asymptote (speedup -> 1/rho as the context grows): under
+    the algorithmic-bytes model the ODA-over-dense ratio rises with t and
+    its gap to 1/rho shrinks like (s + w) / (rho t)."""
+    import bench
+    for rho in (0.125, 0.41):
+        prev = 0.0
+        for t in (4096, 16384, 131072, 524288, 1 << 22):
+            sp = bench.model_speedup(t, rho)
+            assert prev < sp < 1.0 / rho
+            gap = (1.0 / rho - sp) / (1.0 / rho)
+            assert gap <= (2052 + 2) / (rho * t) + 1e-12
+            prev = sp
+    assert abs(bench.model_speedup(524288, 0.125) - 8.0) / 8.0 < 0.04

@@ -386,3 +386,63 @@ def test_smem_limit_never_lowered(torch):
         if r != 2:
             hx.assert_close(st[r], ref["full"], *hx.tol(w), what=f"static row {r}")
     small.close()
+
+
+def test_range_attention(torch):
+    """oda_range_attn (the "<focus>" mode) over [lo, hi) regions of the paged
+    history: the whole history (= Full), regions that start and end inside a
+    block, a single position, a region inside one tile, one from a block
+    boundary to the current token, and one of almost 9000 positions; every
+    listed row and KV head against the oracle. Then a call that lists a
+    subset: unlisted rows keep their output, and regions outside 1..t+1 are
+    reported and leave their row untouched."""
+    from gated_local_full_b200 import oda
+    t0 = (5000, 3000, 700, 2100, 160, 9000)
+    B = len(t0)
+    regions = [(1, 5001), (1000, 2000), (350, 351), (35, 42), (17, 161), (2, 8999)]
+    w = synth.custom("range", hq=16, hkv=8, d=128, window=256, t0=t0, batch=B,
+                     fixed_scores=np.ones(B, np.float32))
+    ctx, dw = hx.setup(w)
+    seq = dw.seq_lens[0]
+    ctx.append_kv(0, 1, dw.k_new[0, 0], dw.v_new[0, 0], seq, dw.block_table, dw.cache, dw.ring,
+                  B)
+    lo = torch.tensor([r[0] for r in regions], dtype=torch.int32, device="cuda")
+    hi = torch.tensor([r[1] for r in regions], dtype=torch.int32, device="cuda")
+    idx = torch.arange(B, dtype=torch.int32, device="cuda")
+    count = torch.full((1,), B, dtype=torch.int32, device="cuda")
+    out = torch.zeros((B, w.hq, w.d), dtype=torch.bfloat16, device="cuda")
+    lse = torch.zeros((B, w.hq), dtype=torch.float32, device="cuda")
+    ctx.range_attn(0, dw.q[0, 0], seq, lo, hi, dw.block_table, dw.cache, idx, count, out, lse, B)
+    torch.cuda.synchronize()
+    assert ctx.get_device_error() == 0
+    q = w.q_step(0)[0]
+    tasks = [(q[b], 0, b, g, regions[b][0], regions[b][1]) for b in range(B)
+             for g in range(w.hkv)]
+    got, got_lse = hx.to_f64(out, w), lse.cpu().numpy().astype(np.float64)
+    for (qb, _, b, g, l_, h_), (o_, lse_) in zip(tasks, hx.oracle_range_heads(w, tasks)):
+        hs = slice(g * w.group, (g + 1) * w.group)
+        hx.assert_close(got[b, hs], o_, *hx.tol(w), what=f"row {b} head {g} [{l_}, {h_})")
+        hx.assert_close(got_lse[b, hs], lse_, 1e-4, 1e-5, what=f"lse row {b} head {g}")
+    # the whole history is Full attention
+    ref = hx.oracle_row(w, 0, 0, 0)
+    hx.assert_close(got[0], ref["full"], *hx.tol(w), what="region = whole history")
+    # a subset of rows, two of them with bad regions
+    before = out.clone()
+    lo2 = lo.clone()
+    hi2 = hi.clone()
+    lo2[1] = 0                               # lo < 1
+    hi2[3] = t0[3] + 2                       # hi > t + 1
+    idx2 = torch.tensor([1, 3, 4, -1, -1, -1], dtype=torch.int32, device="cuda")
+    count2 = torch.full((1,), 3, dtype=torch.int32, device="cuda")
+    hi2[4] = 100
+    ctx.range_attn(0, dw.q[0, 0], seq, lo2, hi2, dw.block_table, dw.cache, idx2, count2, out,
+                   None, B)
+    torch.cuda.synchronize()
+    assert ctx.get_device_error() == oda.ERR_BOUNDS
+    for b in (0, 1, 2, 3, 5):
+        assert torch.equal(out[b], before[b]), f"row {b} changed"
+    (o4, _), = hx.oracle_range_heads(w, [(q[4], 0, 4, 0, 17, 100)])
+    hx.assert_close(hx.to_f64(out, w)[4, 0:2], o4, *hx.tol(w), what="row 4 [17, 100)")
+    with pytest.raises(oda.OdaError):
+        ctx.range_attn(0, dw.q[0, 0], seq, None, hi, dw.block_table, dw.cache, idx, count, out,
+                       None, B)

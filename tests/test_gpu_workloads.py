@@ -172,3 +172,29 @@ def test_run_io_matches_launch_and_copies(torch):
         want = ref["full"] if b != 1 else ref["local"]
         hx.assert_close(out[b], want, *hx.tol(w), what=f"run_io row {b}")
     st.close()
+
+
+def test_full_512k_single_launch(torch):
+    """One Full launch at t = 524288 on a one-layer, 2 GB cache (the pages'
+    512K operating point; 32768 tiles per KV head, so the split, the dynamic
+    tail pool and the 37-partial merges are four times longer than at 128K):
+    every KV head against the oracle, and lse too."""
+    w = synth.ctx128k(steps=1, layers=1, context=524288)
+    ctx, dw = hx.setup(w)
+    seq = dw.seq_lens[0]
+    ctx.append_kv(0, 1, dw.k_new[0], dw.v_new[0], seq, dw.block_table, dw.cache, dw.ring, 1)
+    idx = torch.zeros(1, dtype=torch.int32, device="cuda")
+    count = torch.ones(1, dtype=torch.int32, device="cuda")
+    out = torch.zeros((1, w.hq, w.d), dtype=torch.bfloat16, device="cuda")
+    lse = torch.zeros((1, w.hq), dtype=torch.float32, device="cuda")
+    ctx.full_attn_gated(0, dw.q[0, 0], seq, dw.block_table, dw.cache, idx, count, out, lse, 1)
+    torch.cuda.synchronize()
+    assert ctx.get_device_error() == 0
+    q = w.q_step(0)[0]
+    t = int(w.t0[0])
+    tasks = [(q[0], 0, 0, g, t, True) for g in range(w.hkv)]
+    got, got_lse = hx.to_f64(out, w)[0], lse.cpu().numpy().astype(np.float64)[0]
+    for g, (o, l) in enumerate(hx.oracle_heads(w, tasks)):
+        hs = slice(g * w.group, (g + 1) * w.group)
+        hx.assert_close(got[hs], o, *hx.tol(w), what=f"512K head {g}")
+        hx.assert_close(got_lse[hs], l, 1e-4, 1e-5, what=f"512K lse head {g}")

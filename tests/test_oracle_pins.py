@@ -333,3 +333,67 @@ def test_speedup_tends_to_inverse_rate():
             assert f < prev
         prev = f
     assert abs(prev - 0.125) < 1e-3
+
+
+# --------------------------------------------------------------------------
+# range-restricted ("focus") attention (Declarative Attention pages, the
+# "<focus>" mode: attention narrowed to one region, reading only its KV)
+# --------------------------------------------------------------------------
+
+def test_range_access_set_brute_force():
+    """Position p is in the region [lo, hi) iff lo <= p and p < hi, and the
+    set never reaches outside it."""
+    for lo in range(1, 12):
+        for hi in range(lo, 14):
+            want = {p for p in range(1, 20) if lo <= p < hi}
+            assert o.range_access_set(lo, hi) == want
+            assert len(o.range_access_set(lo, hi)) == hi - lo
+
+
+def test_range_special_cases():
+    """Three regions with a known answer: the whole history is Full, the w
+    most recent positions are Local without sinks, and one position gives
+    its value with lse = its logit."""
+    rng = np.random.default_rng(11)
+    d, t, w = 16, 37, 9
+    q = rng.normal(size=(4, d))
+    K = rng.normal(size=(2, t, d))
+    V = rng.normal(size=(2, t, d))
+    full, lse_f = o.full_attention(q, K, V, t)
+    r, lse_r = o.range_attention(q, K, V, 1, t + 1)
+    assert np.array_equal(full, r) and np.array_equal(lse_f, lse_r)
+    loc, lse_l = o.local_attention(q, K, V, t, 0, w)
+    r, lse_r = o.range_attention(q, K, V, t - w + 1, t + 1)
+    assert np.array_equal(loc, r) and np.array_equal(lse_l, lse_r)
+    p = 13
+    r, lse_r = o.range_attention(q, K, V, p, p + 1)
+    for h in range(4):
+        g = h // 2
+        assert np.allclose(r[h], V[g, p - 1], atol=1e-15)
+        assert abs(lse_r[h] - K[g, p - 1] @ q[h] / math.sqrt(d)) < 1e-12
+
+
+def test_range_two_positions_closed_form():
+    """A region of two positions: the logistic weights of their logit gap,
+    and no weight at all on positions outside it (here a huge-logit key at
+    position 1 that a wrong lower bound would let dominate)."""
+    d = 4
+    q = np.array([[1.0, 0.0, 0.0, 0.0]])
+    K = np.zeros((1, 5, d))
+    K[0, 0, 0] = 100.0            # position 1, outside [3, 5)
+    K[0, 2, 0] = 2.0              # position 3
+    K[0, 3, 0] = -2.0             # position 4
+    K[0, 4, 0] = 100.0            # position 5, outside [3, 5)
+    V = np.zeros((1, 5, d))
+    V[0, 2, 1] = 1.0
+    V[0, 3, 2] = 1.0
+    V[0, 0, 3] = V[0, 4, 3] = 1.0
+    gap = (2.0 - -2.0) / math.sqrt(d)
+    p3 = 1.0 / (1.0 + math.exp(-gap))
+    out, _ = o.range_attention(q, K, V, 3, 5)
+    assert np.allclose(out[0], [0.0, p3, 1.0 - p3, 0.0], atol=1e-15)
+
+
+def test_range_empty_rejected():
+    with pytest.raises(ValueError):
+        o.range_attention(np.zeros((1, 4)), np.zeros((1, 5, 4)), np.zeros((1, 5, 4)), 3, 3)
