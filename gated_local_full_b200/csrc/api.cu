@@ -178,6 +178,12 @@ oda_status oda_create(const oda_config* cfg, oda_ctx** out) {
         cudaMemset(ctx->train_scratch, 0, tb) != cudaSuccess)
       s = ODA_ERR_CUDA;
   }
+  if (s == ODA_OK) {
+    const size_t sb = oda_impl::select_scratch_bytes();
+    if (cudaMalloc(&ctx->select_scratch, sb) != cudaSuccess ||
+        cudaMemset(ctx->select_scratch, 0, sb) != cudaSuccess)
+      s = ODA_ERR_CUDA;
+  }
   if (s == ODA_OK && cudaDeviceSynchronize() != cudaSuccess) s = ODA_ERR_CUDA;
   if (s != ODA_OK) {
     oda_destroy(ctx);
@@ -197,6 +203,7 @@ oda_status oda_destroy(oda_ctx* ctx) {
   cudaFree(ctx->recall_tickets);
   cudaFree(ctx->plan_local);
   cudaFree(ctx->train_scratch);
+  cudaFree(ctx->select_scratch);
   free(ctx);
   return ODA_OK;
 }
@@ -297,6 +304,15 @@ oda_status oda_recall_loss(oda_ctx* ctx, const float* q, const float* logp_full,
   if (n > (int64_t)INT32_MAX) return ODA_ERR_SHAPE;
   return oda_impl::launch_recall_loss(ctx, q, logp_full, logp_local, lambda, (long long)n, loss,
                                       n_full, static_cast<cudaStream_t>(stream));
+}
+
+oda_status oda_select_budget(oda_ctx* ctx, const float* scores, const float* gain, int64_t n,
+                             int64_t k, uint8_t* selected, double* net_gain, oda_stream stream) {
+  if (!ctx || !scores || !selected || n < 1 || k < 0 || k > n) return ODA_ERR_ARG;
+  if (net_gain && !gain) return ODA_ERR_ARG;
+  if (n > (int64_t)INT32_MAX) return ODA_ERR_SHAPE;
+  return oda_impl::launch_select(ctx, scores, gain, (long long)n, (long long)k, selected, net_gain,
+                                 static_cast<cudaStream_t>(stream));
 }
 
 oda_status oda_gate(oda_ctx* ctx, const float* scores, float theta, int B, uint8_t* flags,

@@ -33,6 +33,7 @@ struct oda_ctx {
   int local_wide_cluster_max;  // the same for its one-tile-per-warp shape
   int local_wide_ctas;       // CTAs of that shape one wave holds
   size_t local_last_smem;    // dynamic shared memory of the last Local launch issued
+  void* select_scratch;      // budgeted selection: chunk sums, search state, histogram, counts
 };
 
 // The gate run by the recall head's last CTA inside a captured step.
@@ -49,6 +50,7 @@ struct RecallGate {
 namespace oda {
 
 constexpr int kTrainMaxBlocks = 1024;   // blocks of the recall-loss reduction
+constexpr int kSelectMaxBlocks = 1024;  // blocks (chunks) of the budgeted selection
 
 // ----------------------------------------------------------------- host utils
 #define ODA_CUDA_TRY(expr)                                   \
@@ -252,4 +254,7 @@ oda_status launch_recall_loss(oda_ctx* ctx, const float* q, const float* lpf, co
                               float lam, long long n, float* loss, int32_t* n_full,
                               cudaStream_t st);
 oda_status launch_wait_selftest(oda_ctx* ctx, uint64_t timeout_ns, cudaStream_t st);
+size_t select_scratch_bytes();
+oda_status launch_select(oda_ctx* ctx, const float* scores, const float* gain, long long n,
+                         long long k, uint8_t* selected, double* net_gain, cudaStream_t st);
 }  // namespace oda_impl

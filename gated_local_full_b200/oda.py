@@ -33,7 +33,7 @@ EXPORTS = (
     "oda_get_device_error", "oda_selftest_wait_timeout", "oda_step_run",
     "oda_step_graph_create", "oda_step_graph_launch", "oda_step_graph_run_io",
     "oda_step_graph_destroy", "oda_version",
-    "oda_full_attn_gated_static", "oda_range_attn",
+    "oda_full_attn_gated_static", "oda_range_attn", "oda_select_budget",
 )
 
 
@@ -102,6 +102,7 @@ def lib() -> ctypes.CDLL:
                                        vp, c_int, vp, vp],
         "oda_range_attn": [vp, c_int, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, c_int,
                            ctypes.c_uint, vp],
+        "oda_select_budget": [vp, vp, vp, c_int64, c_int64, vp, vp, vp],
     }
     for name, args in sig.items():
         f = getattr(L, name)
@@ -254,6 +255,16 @@ class OdaContext:
         _check(lib().oda_recall_loss(self.handle, ptr(q), ptr(logp_full), ptr(logp_local),
                                      float(lam), n, ptr(loss), ptr(n_full), _stream(stream)),
                "oda_recall_loss")
+
+    def select_budget(self, scores, gain, k, selected, net_gain=None, stream=None):
+        """The k positions with the largest scores (oda_select_budget), and the
+        net gain per position of that selection when gain is given."""
+        n = scores.numel()
+        if gain is not None and gain.numel() != n:
+            raise ValueError("select_budget: scores and gain differ in length")
+        _check(lib().oda_select_budget(self.handle, ptr(scores), ptr(gain), n, int(k),
+                                       ptr(selected), ptr(net_gain), _stream(stream)),
+               "oda_select_budget")
 
     def gate(self, scores, theta, B, flags, idx, count, stream=None):
         _check(lib().oda_gate(self.handle, ptr(scores), float(theta), B, ptr(flags), ptr(idx),

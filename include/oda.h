@@ -217,13 +217,37 @@ oda_status oda_recall_score(oda_ctx* ctx, const void* h_prev, const void* emb,
  *   q, logp_full, logp_local  device float [n] (recall scores; next-token
  *                             log-probabilities under Full and under Local)
  *   loss     device float [1];  n_full  device int32 [1]
- * The sum is kept in float64 and reduced in a fixed order (deterministic).
+ * The gain, its comparison with lambda and the Huber term are formed in
+ * float64 from the float32 inputs, T's logarithm in float32 (relative error
+ * below 2^-22); the sum is kept in float64 and reduced in a fixed order
+ * (deterministic).
  * 1 <= n <= 2^31 - 1, else ODA_ERR_ARG / ODA_ERR_SHAPE. Uses the context's
  * scratch: calls on one context must not overlap.
  */
 oda_status oda_recall_loss(oda_ctx* ctx, const float* q, const float* logp_full,
                            const float* logp_local, float lambda, int64_t n, float* loss,
                            int32_t* n_full, oda_stream stream);
+
+/*
+ * Selection at a call budget ([SUM] State-Dependent Access Effectiveness: the
+ * net gain a policy captures per reference position at a fixed Full-call
+ * budget, against random selection; Conclusion: the offline Oracle selects by
+ * the true gain). An offline analysis step, not part of a decode step:
+ *   selected[t] = 1 for the k positions with the largest scores, else 0;
+ *     scores compare as float32, equal scores (+0 and -0 alike) go to the
+ *     earlier position, NaN ranks below every number, so the set is unique;
+ *     k = floor(budget * n) is the caller's (0 <= k <= n);
+ *   *net_gain = (1/n) * sum of gain[t] over the selected t (float64, summed
+ *     in a fixed order: the same bits run to run on one GPU).
+ *   scores    device float [n]: the recall head's q_t, or the gain itself for
+ *             the offline Oracle
+ *   gain      device float [n] (access gains g_t), or NULL when net_gain is NULL
+ *   selected  device uint8 [n];  net_gain: device double [1] or NULL
+ * 1 <= n <= 2^31 - 1, else ODA_ERR_ARG / ODA_ERR_SHAPE. Uses the context's
+ * scratch: calls on one context must not overlap.
+ */
+oda_status oda_select_budget(oda_ctx* ctx, const float* scores, const float* gain, int64_t n,
+                             int64_t k, uint8_t* selected, double* net_gain, oda_stream stream);
 
 /*
  * Threshold gate ([SUM] Methodology: recompute with Full iff q_t > theta;

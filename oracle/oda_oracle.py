@@ -17,6 +17,9 @@ Parity status
   delta_F and the FLOP counter ......... pinned (exact integer identity; pages' ratios, loose)
   gelu_erf ............................. pinned (erf closed-form values)
   range_access_set, range_attention .... pinned (brute force, Full/window/one-position cases)
+  budget_count, select_top,
+  net_gain_per_position,
+  random_expected_net_gain ............. pinned (brute force over all k-subsets, closed forms)
   recall_score ......................... parity unpinned: the pages give the
       head's inputs and parameter count but not its architecture; the
       6144 -> 4096 -> 1 GELU MLP is this library's stated choice. Pinned only
@@ -39,6 +42,7 @@ __all__ = [
     "best_action", "regression_target", "attention_flops", "recall_flops",
     "delta_F", "model_step_flops", "oda_flop_fraction",
     "range_access_set", "range_attention",
+    "budget_count", "select_top", "net_gain_per_position", "random_expected_net_gain",
 ]
 
 
@@ -287,6 +291,60 @@ def regression_target(gain, lam: float = 0.0):
     how they combine; placing lambda inside T makes q_t > 0 (the default
     theta) the same decision as best_action, since T is odd and increasing."""
     return signed_log(np.asarray(gain, np.float64) - lam)
+
+
+# ---------------------------------------------------------------------------
+# Selection at a call budget ([SUM] State-Dependent Access Effectiveness: at a
+# 40 % budget the recall head captures a net gain per reference position,
+# compared with the expected gain of random selection; Conclusion: an offline
+# Oracle that knows the true gains selects better still). Readings used (the
+# pages give no formula): a budget b over n positions allows floor(b n) Full
+# calls; a policy spends them on the positions with the largest scores (the
+# recall head's q_t, or the true gain g_t for the offline Oracle), equal
+# scores going to the earlier position and NaN ranking below every number;
+# the net gain per reference position is the sum of g_t over the selected
+# positions divided by n; random selection spends the same calls on a
+# uniformly random subset.
+# ---------------------------------------------------------------------------
+
+def budget_count(n: int, budget) -> int:
+    """Full calls a budget allows: floor(budget * n), in exact arithmetic."""
+    return int(Fraction(budget) * n // 1)
+
+
+def select_top(scores, k: int) -> np.ndarray:
+    """uint8 flags [n]: 1 for the k positions with the largest scores, compared
+    as float32 (equal values, +0 and -0 included, go to the lower position;
+    NaN ranks below every number)."""
+    s = np.asarray(scores, dtype=np.float32)
+    n = s.shape[0]
+    if not 0 <= k <= n:
+        raise ValueError("k outside 0..n")
+
+    def rank_key(i):
+        v = float(s[i])
+        return (1, 0.0, i) if math.isnan(v) else (0, -v, i)
+
+    order = sorted(range(n), key=rank_key)
+    flags = np.zeros(n, dtype=np.uint8)
+    for i in order[:k]:
+        flags[i] = 1
+    return flags
+
+
+def net_gain_per_position(gain, selected) -> float:
+    """(1/n) * sum of g_t over the selected positions."""
+    g = np.asarray(gain, np.float64)
+    sel = np.asarray(selected).astype(bool)
+    return float(g[sel].sum() / g.shape[0])
+
+
+def random_expected_net_gain(gain, k: int) -> float:
+    """Expected net gain per position of k positions drawn uniformly without
+    replacement: each position is drawn with probability k/n."""
+    g = np.asarray(gain, np.float64)
+    n = g.shape[0]
+    return float(k / n * g.sum() / n)
 
 
 # ---------------------------------------------------------------------------

@@ -2,9 +2,9 @@
 against the float64 oracle: mean Huber_1(q - T(g - lambda)) and the count of
 positions whose access gain g = log p^F - log p^L exceeds lambda.
 
-The gain is formed in float32 on the device, so the count is compared
-bit-exactly against the oracle's decision on the same float32 gains; the
-loss, a float64 sum of float32 terms, within 1e-6 + 1e-5 relative."""
+Both sides form the gain f - l and compare it with lambda in float64 from the
+float32 inputs, so the count is compared bit-exactly; the loss (the device
+takes T's logarithm in float32) within 1e-6 + 1e-5 relative."""
 
 import numpy as np
 import pytest
@@ -44,9 +44,9 @@ def _inputs(n, seed, lam):
 
 
 def _oracle(q, lf, ll, lam):
-    g32 = (lf - ll).astype(np.float32)                              # the device's float32 gain
-    y = O.regression_target(g32.astype(np.float64), float(lam))
-    return O.recall_regression_loss(q, y), int(O.best_action(g32, float(lam)).sum())
+    g = O.access_gain(lf, ll)                                       # float64, as the device
+    y = O.regression_target(g, float(lam))
+    return O.recall_regression_loss(q, y), int(O.best_action(g, float(lam)).sum())
 
 
 @pytest.mark.parametrize("n", [1, 7, 1000, 1 << 20, (1 << 20) + 3])

@@ -397,3 +397,53 @@ def test_range_two_positions_closed_form():
 def test_range_empty_rejected():
     with pytest.raises(ValueError):
         o.range_attention(np.zeros((1, 4)), np.zeros((1, 5, 4)), np.zeros((1, 5, 4)), 3, 3)
+
+
+# --------------------------------------------------------------------------
+# selection at a call budget (ODA summary, State-Dependent Access
+# Effectiveness; Conclusion: the offline Oracle)
+# --------------------------------------------------------------------------
+
+def test_budget_count_closed_forms():
+    assert o.budget_count(10, 0.4) == 4
+    assert o.budget_count(7, 0.4) == 2             # floor(2.8)
+    assert o.budget_count(5, 1) == 5 and o.budget_count(5, 0) == 0
+    assert o.budget_count(1000, "0.125") == 125
+
+
+def test_oracle_selection_is_best_and_random_is_the_subset_mean():
+    """Brute force over every k-subset of small gain vectors: selecting by the
+    true gain reaches the largest net gain of any k-subset, and the random
+    expectation is the mean net gain over all k-subsets."""
+    import itertools
+    rng = np.random.default_rng(21)
+    for n in range(1, 8):
+        g = rng.normal(size=n).astype(np.float32)
+        for k in range(0, n + 1):
+            best = max(sum(float(g[i]) for i in c) for c in itertools.combinations(range(n), k))
+            sel = o.select_top(g, k)
+            assert sel.sum() == k
+            assert abs(o.net_gain_per_position(g, sel) - best / n) < 1e-12
+            subsets = list(itertools.combinations(range(n), k))
+            mean = np.mean([sum(float(g[i]) for i in c) / n for c in subsets])
+            assert abs(o.random_expected_net_gain(g, k) - mean) < 1e-12
+
+
+def test_selection_worked_example_and_ties():
+    g = np.array([3.0, -1.0, 2.0, 0.5, -2.0], np.float32)
+    sel = o.select_top(g, 2)
+    assert sel.tolist() == [1, 0, 1, 0, 0]
+    assert o.net_gain_per_position(g, sel) == 1.0
+    assert abs(o.random_expected_net_gain(g, 2) - 0.2) < 1e-15     # 2/5 * 2.5/5
+    # equal scores (+0 and -0 included) go to the earlier position
+    assert o.select_top(np.array([1.0, 1.0, 1.0, 1.0], np.float32), 2).tolist() == [1, 1, 0, 0]
+    assert o.select_top(np.array([-0.0, 0.0, -1.0], np.float32), 1).tolist() == [1, 0, 0]
+    assert o.select_top(np.array([0.0, -0.0, -1.0], np.float32), 1).tolist() == [1, 0, 0]
+    # NaN below every number, -inf included; NaNs among themselves by position
+    s = np.array([np.nan, -np.inf, np.nan, 5.0], np.float32)
+    assert o.select_top(s, 2).tolist() == [0, 1, 0, 1]
+    assert o.select_top(s, 3).tolist() == [1, 1, 0, 1]
+    # the comparison is float32: values equal after rounding tie
+    assert o.select_top(np.array([1.0 + 1e-9, 1.0], np.float64), 1).tolist() == [1, 0]
+    with pytest.raises(ValueError):
+        o.select_top(g, 6)
