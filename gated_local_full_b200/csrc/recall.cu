@@ -648,11 +648,18 @@ recall_cluster_kernel(const __grid_constant__ CUtensorMap tm_w1,
       red[grp * a.B + n] = v;
     }
     __syncthreads();
+    // the groups of each row added by a fixed-order tree (group g takes
+    // g + half while more than one group is left)
+    for (int m = ngrp; m > 1;) {
+      const int half = (m + 1) / 2;
+      for (int i = tid; i < (m - half) * a.B; i += 192)
+        red[i] += red[i + half * a.B];
+      __syncthreads();
+      m = half;
+    }
     if (tid < a.B) {
-      float t2 = 0.f;
-      for (int g2 = 0; g2 < ngrp; ++g2) t2 += red[g2 * a.B + tid];
-      a.scores[tid] = t2 + a.b2;
-      if (warp_gate && own) gval = t2 + a.b2;
+      a.scores[tid] = red[tid] + a.b2;
+      if (warp_gate && own) gval = red[tid] + a.b2;
     }
     if (tid == 0) a.tickets[MAX_MT] = 0;
     if (warp_gate) {
