@@ -921,13 +921,12 @@ attn_kernel(const AttnArgs a) {
     if (nparts > 1) {
       __syncthreads();
       if (tid == 0) {
-        __threadfence();
-        const int prev = atomicAdd(&a.tickets[sigma], 1);
+        const int prev = ticket_add(&a.tickets[sigma], 1);   // releases this CTA's partial
         sflag[0] = (prev == nparts - 1) ? 1 : 0;
       }
       __syncthreads();
       if (sflag[0]) {
-        __threadfence();
+        // (the last ticket acquired every other CTA's partial)
         // Last CTA of the segment: merge its nparts partials. The accumulator
         // loads are issued before the (m, l) reduction so both travel in one
         // L2 round trip.

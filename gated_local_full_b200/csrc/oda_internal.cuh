@@ -179,6 +179,16 @@ __device__ __forceinline__ float fast_log2(float x) {
   return y;
 }
 
+// Ticket increment with acquire-release semantics at GPU scope: the writes
+// the block made before a __syncthreads are released with it, and a block
+// that takes the last ticket acquires every earlier taker's writes (its other
+// threads read them after a __syncthreads), with no separate fences.
+__device__ __forceinline__ int ticket_add(int* p, int v) {
+  int old;
+  asm volatile("atom.add.acq_rel.gpu.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
 // Asynchronous global -> shared copies that hold no registers (cp.async):
 // 16 bytes through L2 only, or 4 bytes; wait_all waits for this thread's.
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {

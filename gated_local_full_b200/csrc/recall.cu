@@ -294,8 +294,7 @@ recall_kernel(const __grid_constant__ CUtensorMap tm_w1, const __grid_constant__
         bool last = true;
         if (nparts > 1) {
           if (tid == 64) {
-            __threadfence();
-            const int prev = atomicAdd(&a.tickets[mt], 1);
+            const int prev = ticket_add(&a.tickets[mt], 1);   // releases this partial
             sflag[0] = (prev == nparts - 1) ? 1 : 0;
           }
           epi_bar();
@@ -303,7 +302,7 @@ recall_kernel(const __grid_constant__ CUtensorMap tm_w1, const __grid_constant__
           epi_bar();
         }
         if (last) {
-          __threadfence();
+          // (the last ticket acquired every other CTA's partial)
           const float bias = a.b1[mt * BM + m];
           const float wo = a.w2[mt * BM + m];
           for (int n0 = 0; n0 < N; n0 += 16) {
@@ -359,13 +358,12 @@ recall_kernel(const __grid_constant__ CUtensorMap tm_w1, const __grid_constant__
           if (tid == 64) a.tickets[mt] = 0;
           epi_bar();
           if (tid == 64) {
-            __threadfence();
-            const int prev = atomicAdd(&a.tickets[MAX_MT], 1);
+            const int prev = ticket_add(&a.tickets[MAX_MT], 1);   // releases the row sums
             sflag[1] = (prev == a.MT - 1) ? 1 : 0;
           }
           epi_bar();
           if (sflag[1]) {
-            __threadfence();
+            // (the last ticket acquired every m-tile's row sums)
             // every (m-tile, row) dot product loaded at once, summed in a
             // fixed order: thread j takes row j % Bc and m-tiles j / Bc + k*step
             const int j = tid - 64;
@@ -615,17 +613,19 @@ recall_cluster_kernel(const __grid_constant__ CUtensorMap tm_w1,
   }
   __syncthreads();
   if (tid == 64) {
-    __threadfence();
-    const int prev = atomicAdd(&a.tickets[MAX_MT], 1);
+    const int prev = ticket_add(&a.tickets[MAX_MT], 1);   // releases this CTA's partials
     sflag[1] = (prev == (int)gridDim.x - 1) ? 1 : 0;
   }
   __syncthreads();
   if (sflag[1]) {
-    __threadfence();
-    // every CTA's partial loaded at once: thread (grp, n) sums CTAs
-    // grp, grp + ngrp, ... of batch row n; the groups are then added in order
-    const int ngrp = 192 / a.B;                           // B <= 64: at least 3 groups
-    const int n = tid % a.B, grp = tid / a.B;
+    // (the ticket acquired every CTA's partial) thread (n, sub) of a group of
+    // TPR lanes, a power of two within one warp, adds CTAs sub, sub + TPR, ...
+    // of batch row n in CTA order; xor shuffles then add the group's lanes in
+    // a fixed order
+    int TPR = 32;
+    while (TPR > 1 && TPR * a.B > 192) TPR >>= 1;
+    const int n = tid / TPR, sub = tid % TPR;
+    const bool row = n < a.B;
     // With at most 32 rows warp 0 gates alone; scores given to the gate from
     // outside are requested together with the partials.
     const bool warp_gate = a.gate_scores != nullptr && a.B <= 32;
@@ -633,34 +633,26 @@ recall_cluster_kernel(const __grid_constant__ CUtensorMap tm_w1,
     float gval = 0.f;
     if (warp_gate && !own && tid < a.B) gval = __ldcg(a.gate_scores + tid);
     float v = 0.f;
-    if (grp < ngrp) {
+    if (row) {
       // eight partials requested at a time, added in CTA order
-      for (int c2 = grp; c2 < (int)gridDim.x; c2 += 8 * ngrp) {
+      for (int c2 = sub; c2 < (int)gridDim.x; c2 += 8 * TPR) {
         float x[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-          const int cc = c2 + u * ngrp;
+          const int cc = c2 + u * TPR;
           x[u] = cc < (int)gridDim.x ? __ldcg(a.spart + (size_t)cc * N + n) : 0.f;
         }
 #pragma unroll
         for (int u = 0; u < 8; ++u) v += x[u];
       }
-      red[grp * a.B + n] = v;
+    }
+    for (int o = 1; o < TPR; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (row && sub == 0) {
+      a.scores[n] = v + a.b2;
+      red[n] = v + a.b2;
     }
     __syncthreads();
-    // the groups of each row added by a fixed-order tree (group g takes
-    // g + half while more than one group is left)
-    for (int m = ngrp; m > 1;) {
-      const int half = (m + 1) / 2;
-      for (int i = tid; i < (m - half) * a.B; i += 192)
-        red[i] += red[i + half * a.B];
-      __syncthreads();
-      m = half;
-    }
-    if (tid < a.B) {
-      a.scores[tid] = red[tid] + a.b2;
-      if (warp_gate && own) gval = red[tid] + a.b2;
-    }
+    if (warp_gate && own && tid < a.B) gval = red[tid];
     if (tid == 0) a.tickets[MAX_MT] = 0;
     if (warp_gate) {
       if (warp == 0)
