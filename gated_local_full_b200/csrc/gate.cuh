@@ -12,6 +12,9 @@
 // The comparison is strict and in float32 (no flush-to-zero: a positive
 // denormal score is above theta = 0); NaN never compares greater. Flagged ids
 // are written in ascending order and the tail of idx is -1.
+//
+// The step graph creates its conditional handle with the default value 0
+// applied at every launch, so the gate sets it only when a row is flagged.
 #pragma once
 
 #include "oda_internal.cuh"
@@ -53,7 +56,7 @@ __device__ __forceinline__ void gate_block(const float* scores, float theta, int
   }
   if (tid == 0) {
     *count = total;
-    if (set_cond) cudaGraphSetConditional(cond, total > 0 ? 1u : 0u);
+    if (set_cond && total > 0) cudaGraphSetConditional(cond, 1u);
   }
 }
 
@@ -74,7 +77,7 @@ __device__ __forceinline__ void gate_warp(float v, int B, float theta, uint8_t* 
   }
   if (lane == 0) {
     *count = total;
-    if (set_cond) cudaGraphSetConditional(cond, total > 0 ? 1u : 0u);
+    if (set_cond && total > 0) cudaGraphSetConditional(cond, 1u);
   }
 }
 

@@ -594,8 +594,11 @@ recall_cluster_kernel(const __grid_constant__ CUtensorMap tm_w1,
     const int TPN = BM / N;                               // threads per batch row
     const int n = j % N, t0 = j / N;
     float s = 0.f;
-    for (int rl = t0; rl < RP; rl += TPN) {               // fixed order
+    // fixed order; unrolled so that the rows' GELU chains overlap
+#pragma unroll 4
+    for (int rl = t0; rl < RP; rl += TPN) {
       float u = 0.f;
+#pragma unroll 4
       for (int r2 = 0; r2 < KS; ++r2) u += rbuf[((size_t)r2 * RP + rl) * N + n];
       s += sw2[rl] * gelu_erf(u + sb1[rl]);
     }
@@ -607,6 +610,7 @@ recall_cluster_kernel(const __grid_constant__ CUtensorMap tm_w1,
     const int TPN = BM / N;
     if (j < N) {
       float s = 0.f;
+#pragma unroll 8
       for (int t2 = 0; t2 < TPN; ++t2) s += red[t2 * N + j];
       a.spart[(size_t)blockIdx.x * N + j] = s;
     }

@@ -131,6 +131,8 @@ oda_status oda_step_graph_create(oda_ctx* ctx, const oda_step_desc* d, oda_graph
     cudaGraph_t cap = nullptr;
     const cudaGraphNode_t* deps = nullptr;
     size_t ndeps = 0;
+    // the condition is 0 at the start of every launch; the gate sets it to 1
+    // when it flags a row
     cudaGraphConditionalHandle handle = 0;
     bool ok = cudaStreamGetCaptureInfo(st, &cs, nullptr, &cap, &deps, &ndeps) == cudaSuccess &&
               cs == cudaStreamCaptureStatusActive &&
