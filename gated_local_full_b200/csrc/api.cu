@@ -201,6 +201,7 @@ oda_status oda_destroy(oda_ctx* ctx) {
   cudaFree(ctx->err);
   cudaFree(ctx->recall_partials);
   cudaFree(ctx->recall_tickets);
+  cudaFree(ctx->recall_pre);
   cudaFree(ctx->plan_local);
   cudaFree(ctx->train_scratch);
   cudaFree(ctx->select_scratch);

@@ -26,6 +26,7 @@ struct oda_ctx {
   int* recall_tickets;       // recall-head split reduction counters
   float* recall_partials;    // recall-head split partials
   int recall_parts_cap;      // capacity of recall_partials in floats
+  float* recall_pre;         // the step's first-layer prefix over h_{t-1}, E(x_t): [hidden][N]
   int recall_cluster_max;    // largest cluster for the recall head's split-K (0: none)
   void* train_scratch;       // recall-loss block sums [kTrainMaxBlocks] f64, counts, ticket
   int* plan_local;           // partition shared by a step's Local launches
@@ -258,7 +259,16 @@ oda_status launch_gate(oda_ctx* ctx, const float* scores, float theta, int B, ui
 oda_status launch_recall(oda_ctx* ctx, const void* h_prev, const void* emb, const void* h_local,
                          int H, const void* W1, const float* b1, const float* w2, float b2,
                          int hidden, float* scores, int B, cudaStream_t st, bool early = false,
-                         const RecallGate* gate = nullptr, bool* gate_fused = nullptr);
+                         const RecallGate* gate = nullptr, bool* gate_fused = nullptr,
+                         bool after_prefix = false);
+// Whether a step splits the head's first layer: the prefix kernel over the
+// K range of h_{t-1} and E(x_t) (launch_recall_prefix, free to run beside the
+// Local launches) and then the cluster kernel over h^L_t only
+// (launch_recall with after_prefix).
+bool recall_split(const oda_ctx* ctx, int B, int H, int hidden);
+oda_status launch_recall_prefix(oda_ctx* ctx, const void* h_prev, const void* emb, int H,
+                                const void* W1, const float* b1, int hidden, int B,
+                                cudaStream_t st);
 oda_status recall_setup(oda_ctx* ctx);
 oda_status launch_recall_loss(oda_ctx* ctx, const float* q, const float* lpf, const float* lpl,
                               float lam, long long n, float* loss, int32_t* n_full,

@@ -62,6 +62,19 @@ struct RecallArgs {
   int32_t* count;
   unsigned long long cond;      // conditional-node handle set from the count, if set_cond
   int set_cond;
+  // Cluster kernel after the step's prefix kernel (pre non-null): K starts at
+  // k-block kb_begin, and pre [KS][hidden][N] (float32) holds the first
+  // layer over k-blocks [0, kb_begin), split in KS quarters, rank r's share
+  // being [r*kb_begin/KS, (r+1)*kb_begin/KS). The prefix's CTAs count
+  // themselves in *pre_done once written; *pre_seen counts those of the
+  // steps before (the last CTA adds MT). A rank that finds this step's
+  // prefix incomplete computes its quarter itself; its owners then add no
+  // prefix for it (nothing waits on the other kernel).
+  int kb_begin;
+  const float* pre;
+  int* pre_done;
+  int* pre_seen;
+  int pre_expected;             // 0: no prefix ran for this call (every rank computes its quarter)
 };
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
@@ -457,7 +470,11 @@ recall_cluster_kernel(const __grid_constant__ CUtensorMap tm_w1,
   const int lane = tid & 31;
   const int rank = (int)blockIdx.x % KS;
   const int mt = (int)blockIdx.x / KS;
-  const int kb0 = (rank * a.KB) / KS, kb1 = ((rank + 1) * a.KB) / KS;
+  const int kspan = a.KB - a.kb_begin;
+  const int kb0 = a.kb_begin + (rank * kspan) / KS, kb1 = a.kb_begin + ((rank + 1) * kspan) / KS;
+  // this rank's quarter of the prefix's K range (computed here only if the
+  // prefix kernel had not finished)
+  const int qb0 = (rank * a.kb_begin) / KS, qb1 = ((rank + 1) * a.kb_begin) / KS;
   const int RP = BM / KS;                                 // rows each rank owns
   uint32_t ncols = 32;
   while ((int)ncols < N) ncols <<= 1;
@@ -470,7 +487,10 @@ recall_cluster_kernel(const __grid_constant__ CUtensorMap tm_w1,
   const int pre = a.early ? min(S, kb1 - kb0) : 0;
   float* sb1 = red + 192;                                 // [RP] b1 of the owned rows
   float* sw2 = sb1 + BM;                                  // [RP] w2 of the owned rows
+  float* sp1 = sw2 + BM;                                  // [KS][RP][N] prefix of the owned rows
+  int* pflag = reinterpret_cast<int*>(sp1 + BM * N);      // [KS] rank r used the prefix
   if (tid == 0) {
+    sflag[3] = 0;                                         // the prefix decision is not made yet
     for (int s2 = 0; s2 < S; ++s2) {
       mbar_init(smem_addr(&full[s2]), 1);
       mbar_init(smem_addr(&empty[s2]), 1);
@@ -507,12 +527,59 @@ recall_cluster_kernel(const __grid_constant__ CUtensorMap tm_w1,
   __syncthreads();
   fence_after_sync();
   const uint32_t tmem = *tmem_slot;
+  // k-blocks: this rank's share of the head's range, then (prefix
+  // incomplete) its quarter of the prefix's range
+  const int n2 = kb1 - kb0;
+  auto kb_at = [&](int i) { return i < n2 ? kb0 + i : qb0 + (i - n2); };
+  // With a prefix, the epilogue warps decide (off the dependency wait's
+  // path; the weights already stream) whether this step's prefix is complete:
+  // once MT more of its CTAs have counted themselves than in the steps before
+  // (acquire: its rows are then visible). If so they load every quarter of the
+  // owned rows' prefix with 16-byte asynchronous copies (each thread waits
+  // for its own before the cluster barrier that precedes their use). The
+  // producer and the MMA issuer read the decision when their share of the
+  // head's range is done (sflag[3] says it is made).
+  bool use_pre = false;
+  if (a.pre && warp >= 2) {
+    if (tid == 64) {
+      int done;
+      asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(done) : "l"(a.pre_done) : "memory");
+      sflag[2] = (a.pre_expected && done - __ldcg(a.pre_seen) >= a.MT) ? 1 : 0;
+      __threadfence_block();
+      *reinterpret_cast<volatile int*>(&sflag[3]) = 1;
+    }
+    epi_bar();
+    use_pre = sflag[2] != 0;
+    if (use_pre) {
+      for (int c = tid - 64; c < BM * N / 4; c += 128) {
+        const int i = 4 * c;
+        const int r2 = i / (RP * N), rem = i - r2 * RP * N;
+        cp_async16(smem_addr(sp1 + i),
+                   a.pre + ((size_t)r2 * a.MT * BM + (size_t)mt * BM + (size_t)rank * RP) * N + rem);
+      }
+    }
+  }
+  // producer / MMA issuer (lane 0): k-blocks after the head's share
+  auto more_kb = [&]() -> int {
+    if (!a.pre) return 0;
+    for (long it = 0; *reinterpret_cast<volatile int*>(&sflag[3]) == 0; ++it) {
+      if (it > (1L << 26)) {                              // bounded: never reached in practice
+        record_error(a.err, ODA_ERR_TIMEOUT);
+        return 0;
+      }
+    }
+    __threadfence_block();
+    return sflag[2] ? 0 : qb1 - qb0;
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
     if (lane == 0) {
       const uint32_t tx = A_STAGE_BYTES + b_stage_bytes;
-      for (int kb = kb0, i = 0; kb < kb1; ++kb, ++i) {
+      int nkb = n2;
+      for (int i = 0; i < nkb; ++i) {
+        if (i == n2 - 1) nkb += more_kb();
+        const int kb = kb_at(i);
         const int s2 = i % S;
         const uint32_t fb = smem_addr(&full[s2]);
         if (i >= pre) {                                   // else W1 was requested early
@@ -535,7 +602,9 @@ recall_cluster_kernel(const __grid_constant__ CUtensorMap tm_w1,
     // ------------------------------------------------------- MMA issuer
     if (lane == 0) {
       const uint32_t idesc = umma_idesc_bf16(N);
-      for (int kb = kb0, i = 0; kb < kb1; ++kb, ++i) {
+      int nkb = n2;
+      for (int i = 0; i < nkb; ++i) {
+        if (i == n2 - 1) nkb += more_kb();
         const int s2 = i % S;
         if (!mbar_wait_bounded(smem_addr(&full[s2]), (uint32_t)((i / S) & 1), kWaitLimitNs)) {
           record_error(a.err, ODA_ERR_TIMEOUT);
@@ -547,7 +616,7 @@ recall_cluster_kernel(const __grid_constant__ CUtensorMap tm_w1,
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk)
           umma_bf16(tmem, ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), idesc,
-                    (kb == kb0 && kk == 0) ? 0u : 1u);
+                    (i == 0 && kk == 0) ? 0u : 1u);
         umma_commit(smem_addr(&empty[s2]));
       }
       umma_commit(smem_addr(acc_full));                   // after every MMA above
@@ -558,9 +627,9 @@ recall_cluster_kernel(const __grid_constant__ CUtensorMap tm_w1,
   namespace cg = cooperative_groups;
   cg::cluster_group cl = cg::this_cluster();
   if (tid == 64) {
-    const bool got = kb0 < kb1 &&
+    const bool got = n2 > 0 &&
                      mbar_wait_bounded(smem_addr(acc_full), 0u, kWaitLimitNs);
-    if (!got && kb0 < kb1) record_error(a.err, ODA_ERR_TIMEOUT);
+    if (!got && n2 > 0) record_error(a.err, ODA_ERR_TIMEOUT);
     sflag[0] = got ? 1 : 0;
   }
   __syncthreads();
@@ -583,12 +652,27 @@ recall_cluster_kernel(const __grid_constant__ CUtensorMap tm_w1,
       for (int e = 0; e < 16; e += 4)
         *reinterpret_cast<float4*>(dst + n0 + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
     }
+    // every owner learns whether this rank's rows include its prefix quarter
+    if (a.pre && tid - 64 < KS) cl.map_shared_rank(pflag, tid - 64)[rank] = use_pre ? 1 : 0;
+    if (use_pre) cp_async_wait_all();                     // this thread's prefix copies
   }
   fence_before_sync();
   cluster_arrive();                                       // release: the pushes
   cluster_wait();                                         // acquire: every rank's pushes
 
   // ------------------------------------- owner: b1, GELU, w2 over its rows
+  if (a.pre && !use_pre && warp >= 2) {
+    // (rare) this rank found the prefix incomplete but another did: that
+    // rank's quarter of the owned rows is read now (the barrier ordered it
+    // after that rank's acquire)
+    for (int i = tid - 64; i < BM * N; i += 128) {
+      const int r2 = i / (RP * N), rem = i - r2 * RP * N;
+      if (pflag[r2])
+        sp1[i] = __ldcg(a.pre + ((size_t)r2 * a.MT * BM + (size_t)mt * BM + (size_t)rank * RP) * N +
+                        rem);
+    }
+    epi_bar();
+  }
   if (warp >= 2) {
     const int j = tid - 64;                               // 0..127
     const int TPN = BM / N;                               // threads per batch row
@@ -599,7 +683,14 @@ recall_cluster_kernel(const __grid_constant__ CUtensorMap tm_w1,
     for (int rl = t0; rl < RP; rl += TPN) {
       float u = 0.f;
 #pragma unroll 4
-      for (int r2 = 0; r2 < KS; ++r2) u += rbuf[((size_t)r2 * RP + rl) * N + n];
+      for (int r2 = 0; r2 < KS; ++r2) {
+        float v = rbuf[((size_t)r2 * RP + rl) * N + n];
+        if (a.pre) {
+          const float p = sp1[((size_t)r2 * RP + rl) * N + n];
+          v += pflag[r2] ? p : 0.f;                       // rank r2's prefix quarter
+        }
+        u += v;
+      }
       s += sw2[rl] * gelu_erf(u + sb1[rl]);
     }
     red[j] = s;
@@ -657,7 +748,10 @@ recall_cluster_kernel(const __grid_constant__ CUtensorMap tm_w1,
     }
     __syncthreads();
     if (warp_gate && own && tid < a.B) gval = red[tid];
-    if (tid == 0) a.tickets[MAX_MT] = 0;
+    if (tid == 0) {
+      a.tickets[MAX_MT] = 0;
+      if (a.pre && a.pre_expected) *a.pre_seen += a.MT;   // this step's prefix is accounted for
+    }
     if (warp_gate) {
       if (warp == 0)
         gate_warp(gval, a.B, a.theta, a.flags, a.idx, a.count, (cudaGraphConditionalHandle)a.cond,
@@ -672,7 +766,146 @@ recall_cluster_kernel(const __grid_constant__ CUtensorMap tm_w1,
   if (warp == 0) {
     __syncwarp();
     // every MMA must have completed before TMEM is released
-    if (kb0 < kb1 && !mbar_wait_bounded(smem_addr(acc_full), 0u, kWaitLimitNs) && lane == 0)
+    if (n2 > 0 && !mbar_wait_bounded(smem_addr(acc_full), 0u, kWaitLimitNs) && lane == 0)
+      record_error(a.err, ODA_ERR_TIMEOUT);
+    __syncwarp();
+    fence_after_sync();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(ncols)
+                 : "memory");
+  }
+}
+
+// The first layer over the K range of h_{t-1} and E(x_t), which are known
+// when a decode step starts (h^L_t only after its last Local launch): one
+// m-tile per CTA over k-blocks [0, kb_end), in KS quarters (the cluster
+// kernel's ranks' shares), each accumulated on its own in TMEM and written
+// to pre [KS][hidden][N] in float32; then the CTA counts itself in
+// *pre_done (release). Sized to run beside the Local launches: four warps
+// (producer, MMA issuer, then all four read one TMEM lane quarter each), two
+// stages, at most 80 registers, so that it fits an SM that holds two Local
+// CTAs.
+__global__ void __launch_bounds__(128, 6)
+recall_prefix_kernel(const __grid_constant__ CUtensorMap tm_w1,
+                     const __grid_constant__ CUtensorMap tm_x0,
+                     const __grid_constant__ CUtensorMap tm_x1, const RecallArgs a, float* pre,
+                     int kb_end, int KS) {
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw = smem_addr(smem_raw);
+  const uint32_t pad = ((raw + 1023u) & ~1023u) - raw;
+  unsigned char* smem = smem_raw + pad;
+  const int S = a.stages;
+  const int N = a.N;
+  const uint32_t b_stage_bytes = (uint32_t)N * BK * 2;
+  unsigned char* sa = smem;
+  unsigned char* sb = sa + (size_t)S * A_STAGE_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sb + (size_t)S * b_stage_bytes);
+  uint64_t* empty = full + S;
+  uint64_t* acc_full = full + 2 * S;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int mt = (int)blockIdx.x;
+  uint32_t ncols = 32;
+  while ((int)ncols < KS * N) ncols <<= 1;
+  if (tid == 0) {
+    for (int s2 = 0; s2 < S; ++s2) {
+      mbar_init(smem_addr(&full[s2]), 1);
+      mbar_init(smem_addr(&empty[s2]), 1);
+    }
+    mbar_init(smem_addr(acc_full), 1);
+    fence_mbar_init();
+  }
+  pdl_wait();
+  if (warp == 0) {
+    __syncwarp();
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_addr(tmem_slot)),
+                 "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  const int m = warp * 32 + lane;                         // row of the m-tile (TMEM lane)
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------ TMA producer
+    const uint32_t tx = A_STAGE_BYTES + b_stage_bytes;
+    for (int kb = 0; kb < kb_end; ++kb) {
+      const int s2 = kb % S;
+      if (!mbar_wait_bounded(smem_addr(&empty[s2]), (uint32_t)(((kb / S) & 1) ^ 1),
+                             kWaitLimitNs)) {
+        record_error(a.err, ODA_ERR_TIMEOUT);
+        break;
+      }
+      const uint32_t fb = smem_addr(&full[s2]);
+      mbar_arrive_expect_tx(fb, tx);
+      tma_load_2d(smem_addr(sa + (size_t)s2 * A_STAGE_BYTES), &tm_w1, kb * BK, mt * BM, fb);
+      const int kglob = kb * BK;
+      const int seg = kglob / a.H;
+      tma_load_2d(smem_addr(sb + (size_t)s2 * b_stage_bytes), seg == 0 ? &tm_x0 : &tm_x1,
+                  kglob - seg * a.H, 0, fb);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------- MMA issuer
+    const uint32_t idesc = umma_idesc_bf16(N);
+    int q = 0, qstart = 0, qnext = kb_end / KS;           // quarter q: [q*kb_end/KS, (q+1)*kb_end/KS)
+    for (int kb = 0; kb < kb_end; ++kb) {
+      while (kb >= qnext) {
+        ++q;
+        qstart = qnext;
+        qnext = ((q + 1) * kb_end) / KS;
+      }
+      const int s2 = kb % S;
+      if (!mbar_wait_bounded(smem_addr(&full[s2]), (uint32_t)((kb / S) & 1), kWaitLimitNs)) {
+        record_error(a.err, ODA_ERR_TIMEOUT);
+        break;
+      }
+      fence_after_sync();
+      const uint64_t ad = umma_desc_sw128(smem_addr(sa + (size_t)s2 * A_STAGE_BYTES));
+      const uint64_t bd = umma_desc_sw128(smem_addr(sb + (size_t)s2 * b_stage_bytes));
+#pragma unroll
+      for (int kk = 0; kk < BK / 16; ++kk)
+        umma_bf16(tmem + (uint32_t)(q * N), ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk),
+                  idesc, (kb == qstart && kk == 0) ? 0u : 1u);
+      umma_commit(smem_addr(&empty[s2]));
+    }
+    umma_commit(smem_addr(acc_full));                     // after every MMA above
+  }
+  __syncwarp();
+  // ---------------------------------------- epilogue: one lane quarter per warp
+  const bool got = __all_sync(0xffffffffu, kb_end > 0 && mbar_wait_bounded(smem_addr(acc_full),
+                                                                              0u, kWaitLimitNs));
+  if (!got && kb_end > 0 && lane == 0) record_error(a.err, ODA_ERR_TIMEOUT);
+  fence_after_sync();
+  for (int q = 0; q < KS; ++q) {
+    float* dst = pre + ((size_t)q * a.MT * BM + (size_t)mt * BM + m) * N;
+    for (int n0 = 0; n0 < N; n0 += 16) {
+      float v[16];
+      if (got) {
+        tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(q * N + n0), v);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) v[e] = 0.f;
+      }
+#pragma unroll
+      for (int e = 0; e < 16; e += 4)
+        *reinterpret_cast<float4*>(dst + n0 + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+    }
+  }
+  fence_before_sync();
+  __syncthreads();
+  // every row written: count this CTA (release; a timed-out CTA does not)
+  if (tid == 0 && got)
+    asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(a.pre_done) : "memory");
+  if (warp == 0) {
+    // every MMA must have completed before TMEM is released
+    if (kb_end > 0 && !got && !mbar_wait_bounded(smem_addr(acc_full), 0u, kWaitLimitNs) &&
+        lane == 0)
       record_error(a.err, ODA_ERR_TIMEOUT);
     __syncwarp();
     fence_after_sync();
@@ -727,25 +960,48 @@ size_t smem_for(int n, int s) {
          4 * MAX_N * 4 + 64;
 }
 
-// Stages and shared memory of the cluster kernel (its row buffer comes first).
-int cl_stages_for(int n) {
-  const int per = A_STAGE_BYTES + n * BK * 2;
-  int s = (200 * 1024 - BM * n * 4) / per;
-  if (s > 8) s = 8;
-  if (s < 2) s = 2;
-  return s;
+// Shared memory of the cluster kernel with s stages (its row buffer comes first).
+size_t cl_smem_for(int n, int s, size_t extra = 0) {
+  return 1024 + (size_t)s * (A_STAGE_BYTES + n * BK * 2) + (size_t)(2 * s + 1) * 8 + 4 + 16 + 16 +
+         (size_t)(BM * n + 192 + 2 * BM) * 4 + extra + 64;
 }
 
-size_t cl_smem_for(int n, int s) {
-  return 1024 + (size_t)s * (A_STAGE_BYTES + n * BK * 2) + (size_t)(2 * s + 1) * 8 + 4 + 16 + 16 +
-         (size_t)(BM * n + 192 + 2 * BM) * 4 + 64;
-}
+// `extra` after the prefix kernel: every quarter of the owned rows' prefix
+// (KS * 128/KS * n floats) and the ranks' flags
+size_t cl_pre_bytes(int n) { return (size_t)BM * n * 4 + 64; }
+
+// The cluster kernel's shared-memory limit: the most one CTA may have.
+constexpr size_t kClusterSmemMax = 227 * 1024;
 
 // Stages of the cluster kernel within `budget` bytes of shared memory.
-int cl_stages_within(int n, size_t budget) {
+int cl_stages_within(int n, size_t budget, size_t extra) {
   int s = 8;
-  while (s > 2 && cl_smem_for(n, s) > budget) --s;
+  while (s > 2 && cl_smem_for(n, s, extra) > budget) --s;
   return s;
+}
+
+// The prefix kernel: two stages (it runs beside two Local CTAs).
+#ifndef ODA_PREFIX_STAGES
+#define ODA_PREFIX_STAGES 2
+#endif
+constexpr int kPrefixStages = ODA_PREFIX_STAGES;
+size_t prefix_smem_for(int n) {
+  return 1024 + (size_t)kPrefixStages * (A_STAGE_BYTES + n * BK * 2) +
+         (size_t)(2 * kPrefixStages + 1) * 8 + 4 + 64;
+}
+
+// Cluster size of the split-K kernel for batch width N, or 0 for the
+// stream-K kernel: every m-tile gets a whole cluster within one wave.
+int cluster_ks(const oda_ctx* ctx, int N, int MT, int KB) {
+  if (N != 16 && N != 32 && N != 64) return 0;
+  for (int ks = ctx->recall_cluster_max; ks >= 2; ks >>= 1)
+    if (MT * ks <= ctx->num_sms && KB >= ks) return ks;
+  return 0;
+}
+
+bool shape_ok(int B, int H, int hidden) {
+  return B >= 1 && B <= MAX_N && H >= BK && H % BK == 0 && hidden >= BM && hidden % BM == 0 &&
+         hidden / BM <= MAX_MT;
 }
 
 }  // namespace
@@ -760,11 +1016,18 @@ oda_status recall_setup(oda_ctx* ctx) {
   const size_t pfl = (size_t)(ctx->num_sms + MAX_MT) * MAX_N * BM + (size_t)MAX_MT * MAX_N;
   ODA_CUDA_TRY(cudaMalloc(&ctx->recall_partials, pfl * sizeof(float)));
   ctx->recall_parts_cap = (int)((size_t)(ctx->num_sms + MAX_MT) * MAX_N * BM);
-  ODA_CUDA_TRY(cudaMalloc(&ctx->recall_tickets, (MAX_MT + 1) * sizeof(int)));
-  ODA_CUDA_TRY(cudaMemset(ctx->recall_tickets, 0, (MAX_MT + 1) * sizeof(int)));
+  // tickets: [MAX_MT] per m-tile, [MAX_MT] the final sum, then the prefix's
+  // done and seen counters
+  ODA_CUDA_TRY(cudaMalloc(&ctx->recall_tickets, (MAX_MT + 3) * sizeof(int)));
+  ODA_CUDA_TRY(cudaMemset(ctx->recall_tickets, 0, (MAX_MT + 3) * sizeof(int)));
+  // the prefix: [KS][hidden][N] with KS * hidden / 128 <= SMs
+  ODA_CUDA_TRY(cudaMalloc(&ctx->recall_pre,
+                          (size_t)ctx->num_sms * BM * CL_MAX_N * sizeof(float)));
+  ODA_CUDA_TRY(raise_smem_limit(reinterpret_cast<const void*>(recall_prefix_kernel),
+                                prefix_smem_for(CL_MAX_N)));
   // the cluster split-K kernel: the largest cluster (8, 4, 2) the GPU holds
   ctx->recall_cluster_max = 0;
-  const size_t csm = cl_smem_for(CL_MAX_N, cl_stages_for(CL_MAX_N));
+  const size_t csm = kClusterSmemMax;
   if (raise_smem_limit(reinterpret_cast<const void*>(recall_cluster_kernel), csm) ==
       cudaSuccess) {
     for (int ks = 8; ks >= 2; ks >>= 1) {
@@ -794,11 +1057,11 @@ oda_status recall_setup(oda_ctx* ctx) {
 oda_status launch_recall(oda_ctx* ctx, const void* h_prev, const void* emb, const void* h_local,
                          int H, const void* W1, const float* b1, const float* w2, float b2,
                          int hidden, float* scores, int B, cudaStream_t st, bool early,
-                         const RecallGate* gate, bool* gate_fused) {
+                         const RecallGate* gate, bool* gate_fused, bool after_prefix) {
   if (gate_fused) *gate_fused = false;
-  if (B < 1 || B > MAX_N || H < BK || H % BK != 0 || hidden < BM || hidden % BM != 0 ||
-      hidden / BM > MAX_MT)
-    return ODA_ERR_SHAPE;
+  if (!shape_ok(B, H, hidden)) return ODA_ERR_SHAPE;
+  const bool split = recall_split(ctx, B, H, hidden);
+  if (after_prefix && !split) return ODA_ERR_SHAPE;
   const int N = ((B + 15) / 16) * 16;
   CUtensorMap tw, t0, t1, t2;
   const uint64_t K = 3ull * (uint64_t)H;
@@ -828,22 +1091,27 @@ oda_status launch_recall(oda_ctx* ctx, const void* h_prev, const void* emb, cons
   a.count = nullptr;
   a.cond = 0ull;
   a.set_cond = 0;
+  // Where the step splits the head, every call runs the split layout: after
+  // the step's prefix kernel, or alone with every rank computing its quarter
+  // of the prefix's range itself.
+  a.kb_begin = split ? 2 * H / BK : 0;
+  a.pre = split ? ctx->recall_pre : nullptr;
+  a.pre_done = ctx->recall_tickets + MAX_MT + 1;
+  a.pre_seen = ctx->recall_tickets + MAX_MT + 2;
+  a.pre_expected = after_prefix ? 1 : 0;
   // cluster split-K when every m-tile gets a whole cluster within one wave
-  int KS = 0;
-  if (N == 16 || N == 32 || N == 64) {
-    for (int ks = ctx->recall_cluster_max; ks >= 2; ks >>= 1)
-      if (a.MT * ks <= ctx->num_sms && a.KB >= ks) { KS = ks; break; }
-  }
+  const int KS = cluster_ks(ctx, N, a.MT, a.KB - a.kb_begin);
   if (KS >= 2) {
-    a.stages = cl_stages_for(N);
+    const size_t extra = split ? cl_pre_bytes(N) : 0;
+    a.stages = cl_stages_within(N, kClusterSmemMax, extra);
     if (early) {
       // The CTAs are to become resident beside the preceding Local launch's
       // CTAs (one per SM) and request W1 while it runs: fewer stages, so both
       // fit one SM's shared memory (1 KB of it is reserved per CTA).
       const size_t sm_total = 228 * 1024;
       const size_t beside = ctx->local_last_smem + 2 * 1024;
-      if (ctx->local_last_smem > 0 && beside + cl_smem_for(N, 2) <= sm_total)
-        a.stages = cl_stages_within(N, sm_total - beside);
+      if (ctx->local_last_smem > 0 && beside + cl_smem_for(N, 2, extra) <= sm_total)
+        a.stages = cl_stages_within(N, sm_total - beside, extra);
       a.early = 1;
     }
     if (gate && B <= 192) {
@@ -858,7 +1126,7 @@ oda_status launch_recall(oda_ctx* ctx, const void* h_prev, const void* emb, cons
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(a.MT * KS);
     cfg.blockDim = dim3(192);
-    cfg.dynamicSmemBytes = cl_smem_for(N, a.stages);
+    cfg.dynamicSmemBytes = cl_smem_for(N, a.stages, extra);
     cfg.stream = st;
     cudaLaunchAttribute at[2];
     at[0].id = cudaLaunchAttributeClusterDimension;
@@ -879,6 +1147,40 @@ oda_status launch_recall(oda_ctx* ctx, const void* h_prev, const void* emb, cons
   const int grid = U < ctx->num_sms ? U : ctx->num_sms;
   return launch_pdl(recall_kernel, dim3(grid), dim3(192), smem_for(N, a.stages), st, tw, t0, t1,
                     t2, a) == cudaSuccess
+             ? ODA_OK
+             : ODA_ERR_CUDA;
+}
+
+bool recall_split(const oda_ctx* ctx, int B, int H, int hidden) {
+  if (!shape_ok(B, H, hidden)) return false;
+  const int N = ((B + 15) / 16) * 16;
+  const int MT = hidden / BM;
+  const int ks = cluster_ks(ctx, N, MT, H / BK);         // the cluster kernel's K: h^L_t
+  return ks >= 2 && cluster_ks(ctx, N, MT, 3 * H / BK) == ks;
+}
+
+oda_status launch_recall_prefix(oda_ctx* ctx, const void* h_prev, const void* emb, int H,
+                                const void* W1, const float* b1, int hidden, int B,
+                                cudaStream_t st) {
+  if (!recall_split(ctx, B, H, hidden)) return ODA_ERR_SHAPE;
+  const int N = ((B + 15) / 16) * 16;
+  CUtensorMap tw, t0, t1;
+  if (!encode_2d(&tw, W1, 3ull * (uint64_t)H, (uint64_t)hidden, BK, BM)) return ODA_ERR_CUDA;
+  if (!encode_2d(&t0, h_prev, (uint64_t)H, (uint64_t)B, BK, (uint32_t)N)) return ODA_ERR_CUDA;
+  if (!encode_2d(&t1, emb, (uint64_t)H, (uint64_t)B, BK, (uint32_t)N)) return ODA_ERR_CUDA;
+  RecallArgs a = {};
+  a.b1 = b1;
+  a.err = ctx->err;
+  a.B = B;
+  a.N = N;
+  a.MT = hidden / BM;
+  a.KB = 3 * H / BK;
+  a.H = H;
+  a.stages = kPrefixStages;
+  a.pre_done = ctx->recall_tickets + MAX_MT + 1;
+  const int KS = cluster_ks(ctx, N, a.MT, H / BK);       // the cluster kernel's ranks
+  return launch_pdl(recall_prefix_kernel, dim3(a.MT), dim3(128), prefix_smem_for(N), st, tw, t0,
+                    t1, a, ctx->recall_pre, 2 * H / BK, KS) == cudaSuccess
              ? ODA_OK
              : ODA_ERR_CUDA;
 }

@@ -43,13 +43,38 @@ size_t layer_elems(const oda_ctx* ctx, int B, int heads) {
 // its predecessor before it lets the next launch start. So from the second
 // launch of each kind on, the inputs a launch stages before its own
 // dependency wait were complete before it started.
-oda_status pre_part(oda_ctx* ctx, const oda_step_desc* d, cudaStream_t st,
-                    unsigned long long cond, bool set_cond) {
+//
+// The recall head reads h_{t-1} and E(x_t), inputs of the step, and h^L_t,
+// known only after the last Local launch. Where the head splits (recall_split),
+// its first layer over the first two runs as a kernel of its own that starts
+// with the step: on `side` (a captured graph), forked from `st` at the start,
+// so that its weight stream overlaps the Local launches (which leave most of
+// the memory bandwidth unused); without a side stream it runs first. The rest
+// of the head then streams only the weights of h^L_t. No graph edge joins the
+// prefix to the head: an edge from another branch would hold the head's
+// launch past the last Local launch's completion, and its first weight tiles
+// could no longer be requested while that launch runs. The prefix counts its
+// finished CTAs instead, and each rank of the head that finds it incomplete
+// computes its own share of the prefix's range. The side stream rejoins
+// `st` after the head (before the conditional node).
+oda_status pre_part(oda_ctx* ctx, const oda_step_desc* d, cudaStream_t st, cudaStream_t side,
+                    cudaEvent_t fork, cudaEvent_t join, unsigned long long cond, bool set_cond) {
   const oda_config& c = ctx->cfg;
   const size_t eb = (size_t)ctx->lay.elem_bytes;
-  oda_status s = oda_impl::launch_append(ctx, 0, c.layers, d->k_new, d->v_new, d->seq_lens,
-                                         d->block_table, d->kv_cache, d->ring, d->B, st,
-                                         ctx->plan_local);
+  oda_status s = ODA_OK;
+  const bool split = d->W1 && oda_impl::recall_split(ctx, d->B, d->H, d->hidden);
+  if (split) {
+    if (side) {
+      if (cudaEventRecord(fork, st) != cudaSuccess || cudaStreamWaitEvent(side, fork, 0) != cudaSuccess)
+        return ODA_ERR_CUDA;
+    }
+    s = oda_impl::launch_recall_prefix(ctx, d->h_prev, d->emb, d->H, d->W1, d->b1, d->hidden,
+                                       d->B, side ? side : st);
+    if (s != ODA_OK) return s;
+    if (side && cudaEventRecord(join, side) != cudaSuccess) return ODA_ERR_CUDA;
+  }
+  s = oda_impl::launch_append(ctx, 0, c.layers, d->k_new, d->v_new, d->seq_lens, d->block_table,
+                              d->kv_cache, d->ring, d->B, st, ctx->plan_local);
   if (s != ODA_OK) return s;
   for (int l = 0; l < c.layers; ++l) {
     const size_t qo = (size_t)l * layer_elems(ctx, d->B, c.hq) * eb;
@@ -75,8 +100,10 @@ oda_status pre_part(oda_ctx* ctx, const oda_step_desc* d, cudaStream_t st,
     g.cond = cond;
     g.set_cond = set_cond;
     s = oda_impl::launch_recall(ctx, d->h_prev, d->emb, d->h_local, d->H, d->W1, d->b1, d->w2,
-                                d->b2, d->hidden, d->scores, d->B, st, /*early=*/true, &g, &gated);
+                                d->b2, d->hidden, d->scores, d->B, st, /*early=*/true, &g, &gated,
+                                /*after_prefix=*/split);
     if (s != ODA_OK) return s;
+    if (split && side && cudaStreamWaitEvent(st, join, 0) != cudaSuccess) return ODA_ERR_CUDA;
   }
   if (gated) return ODA_OK;
   return oda_impl::launch_gate(ctx, gs, d->theta, d->B, d->flags, d->idx, d->count, st, cond,
@@ -106,7 +133,7 @@ oda_status oda_step_run(oda_ctx* ctx, const oda_step_desc* d, oda_stream stream)
   oda_status s = check_desc(ctx, d);
   if (s != ODA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  s = pre_part(ctx, d, st, 0ull, false);
+  s = pre_part(ctx, d, st, nullptr, nullptr, nullptr, 0ull, false);
   if (s != ODA_OK) return s;
   return full_part(ctx, d, st);
 }
@@ -116,16 +143,18 @@ oda_status oda_step_graph_create(oda_ctx* ctx, const oda_step_desc* d, oda_graph
   *out = nullptr;
   oda_status s = check_desc(ctx, d);
   if (s != ODA_OK) return s;
-  cudaStream_t st = nullptr, st2 = nullptr;
+  cudaStream_t st = nullptr, st2 = nullptr, st3 = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
   cudaGraph_t graph = nullptr;
   cudaGraphExec_t exec = nullptr;
-  ODA_CUDA_TRY(cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking));
-  if (cudaStreamCreateWithFlags(&st2, cudaStreamNonBlocking) != cudaSuccess) {
-    cudaStreamDestroy(st);
-    return ODA_ERR_CUDA;
-  }
   s = ODA_ERR_CUDA;
   do {
+    if (cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&st2, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&st3, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&join, cudaEventDisableTiming) != cudaSuccess)
+      break;
     if (cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal) != cudaSuccess) break;
     cudaStreamCaptureStatus cs;
     cudaGraph_t cap = nullptr;
@@ -138,7 +167,8 @@ oda_status oda_step_graph_create(oda_ctx* ctx, const oda_step_desc* d, oda_graph
               cs == cudaStreamCaptureStatusActive &&
               cudaGraphConditionalHandleCreate(&handle, cap, 0, cudaGraphCondAssignDefault) ==
                   cudaSuccess;
-    oda_status ps = ok ? pre_part(ctx, d, st, (unsigned long long)handle, true) : ODA_ERR_CUDA;
+    oda_status ps =
+        ok ? pre_part(ctx, d, st, st3, fork, join, (unsigned long long)handle, true) : ODA_ERR_CUDA;
     cudaGraphNode_t cond_node = nullptr;
     cudaGraph_t body = nullptr;
     if (ps == ODA_OK &&
@@ -180,11 +210,23 @@ oda_status oda_step_graph_create(oda_ctx* ctx, const oda_step_desc* d, oda_graph
       graph = nullptr;
       break;
     }
+    // upload now, so that the first launch does not pay for it (its
+    // branches then start together, like every later launch's)
+    if (cudaGraphUpload(exec, st) != cudaSuccess || cudaStreamSynchronize(st) != cudaSuccess) {
+      cudaGraphExecDestroy(exec);
+      cudaGraphDestroy(graph);
+      graph = nullptr;
+      exec = nullptr;
+      break;
+    }
     s = ODA_OK;
   } while (false);
   cudaGetLastError();
-  cudaStreamDestroy(st);
-  cudaStreamDestroy(st2);
+  if (join) cudaEventDestroy(join);
+  if (fork) cudaEventDestroy(fork);
+  if (st3) cudaStreamDestroy(st3);
+  if (st2) cudaStreamDestroy(st2);
+  if (st) cudaStreamDestroy(st);
   if (s != ODA_OK) return s;
   oda_graph* g = static_cast<oda_graph*>(calloc(1, sizeof(oda_graph)));
   if (!g) {

@@ -370,14 +370,23 @@ typedef struct oda_step_desc {
 
 /* Issue one step with plain launches: append (all layers, one launch), Local
  * per layer, recall head, gate, then Full per layer (those kernels exit at
- * once when *count == 0). */
+ * once when *count == 0). Where the head's shape allows (batch <= 64 and its
+ * m-tiles times a cluster fit the SMs), its first layer over h_prev and emb,
+ * inputs of the step, runs as a kernel of its own before the append; the
+ * rest of the head, after the last Local launch, streams the weights of
+ * h_local only. */
 oda_status oda_step_run(oda_ctx* ctx, const oda_step_desc* d, oda_stream stream);
 
 /* Capture the same step as a CUDA graph in which the Full launches sit in the
  * body of a conditional IF node that the gate kernel sets from *count, so a
  * step with no flagged row launches no Full kernel ([SUM] Efficient
- * Execution: GPU-side conditional CUDA Graphs). The descriptor's pointers are
- * baked in: refill the same buffers between launches. */
+ * Execution: GPU-side conditional CUDA Graphs). The head's first-layer part
+ * over h_prev and emb is a branch of its own that starts with the graph and
+ * runs beside the Local launches; the rest of the head does not wait for it
+ * (a rank of it that finds that part unfinished computes its own share of it
+ * instead), so scores can differ between launches in float32 rounding only.
+ * The descriptor's pointers are baked in: refill the same buffers between
+ * launches. */
 oda_status oda_step_graph_create(oda_ctx* ctx, const oda_step_desc* d, oda_graph** out);
 oda_status oda_step_graph_launch(oda_graph* g, oda_stream stream);
 

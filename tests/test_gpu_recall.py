@@ -133,3 +133,41 @@ def test_gated_step_with_recall_head(torch, ctxlen):
         hx.assert_close(out[b, g * w.group:(g + 1) * w.group], o, *hx.tol(w),
                         what=f"row {b} head {g}")
     st.close()
+
+
+def test_step_recall_split_plain_and_graph(torch):
+    """The step splits the head's first layer: h_{t-1} and E(x_t) in a kernel
+    that starts with the step (beside the Local launches in the graph, first
+    on one stream otherwise), h^L_t after the last Local launch. A rank of the
+    head that finds the prefix incomplete computes its share of the prefix's
+    range itself, so the sum order (not the result) can differ between runs:
+    both stay within the head's tolerance of the oracle and agree to float32
+    rounding. On one stream the prefix is always complete, so repeated plain
+    steps agree bit for bit."""
+    from gated_local_full_b200.runtime import DecodeStep
+    w = synth.recall_step(4096)
+    ctx, dw = hx.setup(w)
+    r = dw.recall
+    got = []
+    for graph in (False, True, False, True):
+        st = DecodeStep(ctx, w.batch, dw.cache, dw.ring, dw.block_table, recall=r, graph=graph)
+        st.feed(dw.q[0], dw.k_new[0], dw.v_new[0], dw.seq_lens[0], h_prev=r["h_prev"][0],
+                emb=r["emb"][0], h_local=r["h_local"][0])
+        st.run()
+        torch.cuda.synchronize()
+        assert ctx.get_device_error() == 0
+        got.append(st.scores.cpu().numpy().astype(np.float64))
+        st.close()
+    assert np.array_equal(got[0], got[2])
+    ref = _recall_oracle(w)
+    for g in got:
+        hx.assert_close(g, ref, SCORE_ATOL, SCORE_RTOL, "scores")
+        np.testing.assert_allclose(g, got[0], rtol=1e-5, atol=1e-5)
+    # the standalone head: every rank computes its quarter of the prefix's range
+    s = torch.empty(w.batch, dtype=torch.float32, device="cuda")
+    ctx.recall_score(r["h_prev"][0], r["emb"][0], r["h_local"][0], r["H"], r["W1"], r["b1"],
+                     r["w2"], r["b2"], r["hidden"], s, w.batch)
+    torch.cuda.synchronize()
+    alone = s.cpu().numpy().astype(np.float64)
+    hx.assert_close(alone, ref, SCORE_ATOL, SCORE_RTOL, "standalone scores")
+    np.testing.assert_allclose(alone, got[0], rtol=1e-5, atol=1e-5)
