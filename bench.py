@@ -762,11 +762,13 @@ def run_oda(args, rank, ws, local):
         launches = K * (w.layers + 1)
     else:
         kv_bytes = sum(batch_step_bytes(w, j, flags[j]) for j in recs_timed)
-        # append, Local x L, the recall head (its last CTA gates), then Full x L:
-        # behind the IF node only steps with a flagged row launch them; plain
-        # launches issue the gate and the Full launches every step
+        # the recall head's prefix kernel (its first layer over h_{t-1} and
+        # E(x_t); every workload here is a shape the step splits), append,
+        # Local x L, the rest of the recall head (its last CTA gates), then
+        # Full x L: behind the IF node only steps with a flagged row launch
+        # them; plain launches issue the Full launches every step
         if args.launch == "graph":
-            launches = K * (w.layers + 2) + n_flag_steps * w.layers
+            launches = K * (w.layers + 3) + n_flag_steps * w.layers
         else:
             launches = K * (2 * w.layers + 3)
 
