@@ -763,14 +763,16 @@ def run_oda(args, rank, ws, local):
     else:
         kv_bytes = sum(batch_step_bytes(w, j, flags[j]) for j in recs_timed)
         # the recall head's prefix kernel (its first layer over h_{t-1} and
-        # E(x_t); every workload here is a shape the step splits), append,
-        # Local x L, the rest of the recall head (its last CTA gates), then
-        # Full x L: behind the IF node only steps with a flagged row launch
-        # them; plain launches issue the Full launches every step
+        # E(x_t), in steps of enough layers; every workload here has a head
+        # shape the step splits), append, Local x L, the rest of the recall
+        # head (its last CTA gates), then Full x L: behind the IF node only
+        # steps with a flagged row launch them; plain launches issue the Full
+        # launches every step
+        pre = 1 if w.layers >= oda.RECALL_SPLIT_MIN_LAYERS else 0
         if args.launch == "graph":
-            launches = K * (w.layers + 3) + n_flag_steps * w.layers
+            launches = K * (w.layers + 2 + pre) + n_flag_steps * w.layers
         else:
-            launches = K * (2 * w.layers + 3)
+            launches = K * (2 * w.layers + 2 + pre)
 
     # ---- per-kernel launch times, as in a step: the L layers' launches back
     # to back (flag set from the second on), for up to 16 timed steps, each on

@@ -35,6 +35,9 @@ size_t layer_elems(const oda_ctx* ctx, int B, int heads) {
   return (size_t)B * heads * ctx->cfg.head_dim;
 }
 
+// The step splits the recall head only above this many layers.
+constexpr int kRecallSplitMinLayers = 8;
+
 // Early staging (launch_attn's `early`): the append kernel writes the ring
 // and the paged cache of every layer, the record copy before it holds the
 // lengths, and the gate writes the compacted ids. Every Local launch after the
@@ -62,7 +65,10 @@ oda_status pre_part(oda_ctx* ctx, const oda_step_desc* d, cudaStream_t st, cudaS
   const oda_config& c = ctx->cfg;
   const size_t eb = (size_t)ctx->lay.elem_bytes;
   oda_status s = ODA_OK;
-  const bool split = d->W1 && oda_impl::recall_split(ctx, d->B, d->H, d->hidden);
+  // (the prefix takes ~40 us beside the Local launches; with fewer layers the
+  // head would find it unfinished and both would stream its weights)
+  const bool split = d->W1 && c.layers >= kRecallSplitMinLayers &&
+                     oda_impl::recall_split(ctx, d->B, d->H, d->hidden);
   if (split) {
     if (side) {
       if (cudaEventRecord(fork, st) != cudaSuccess || cudaStreamWaitEvent(side, fork, 0) != cudaSuccess)

@@ -23,6 +23,9 @@ OK, ERR_ARG, ERR_SHAPE, ERR_DTYPE, ERR_CUDA, ERR_TIMEOUT, ERR_BOUNDS, ERR_STATE 
 BF16, F32 = 0, 1
 MAX_BATCH = 1024
 ATTN_INPUTS_READY = 1     # oda_local_attn / oda_full_attn_gated flag (see oda.h)
+# A step with at least this many layers runs the recall head's first layer over
+# h_prev and emb as a kernel of its own (oda.h, oda_step_run): one launch more.
+RECALL_SPLIT_MIN_LAYERS = 8
 STATUS_NAMES = {0: "ODA_OK", 1: "ODA_ERR_ARG", 2: "ODA_ERR_SHAPE", 3: "ODA_ERR_DTYPE",
                 4: "ODA_ERR_CUDA", 5: "ODA_ERR_TIMEOUT", 6: "ODA_ERR_BOUNDS", 7: "ODA_ERR_STATE"}
 

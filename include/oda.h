@@ -370,8 +370,9 @@ typedef struct oda_step_desc {
 
 /* Issue one step with plain launches: append (all layers, one launch), Local
  * per layer, recall head, gate, then Full per layer (those kernels exit at
- * once when *count == 0). Where the head's shape allows (batch <= 64 and its
- * m-tiles times a cluster fit the SMs), its first layer over h_prev and emb,
+ * once when *count == 0). With 8 layers or more, where the head's shape
+ * allows (batch <= 64 and its m-tiles times a cluster fit the SMs), its
+ * first layer over h_prev and emb,
  * inputs of the step, runs as a kernel of its own before the append; the
  * rest of the head, after the last Local launch, streams the weights of
  * h_local only. */

@@ -145,7 +145,10 @@ def test_step_recall_split_plain_and_graph(torch):
     rounding. On one stream the prefix is always complete, so repeated plain
     steps agree bit for bit."""
     from gated_local_full_b200.runtime import DecodeStep
-    w = synth.recall_step(4096)
+    from gated_local_full_b200 import oda
+    # a step of enough layers for the split (batch 16, hidden 2048, 6144 -> 4096)
+    w = synth.custom("recall_split", layers=oda.RECALL_SPLIT_MIN_LAYERS, batch=16, t0=[300],
+                     hq=16, hkv=8, window=128, recall=True, hidden=2048, recall_hidden=4096)
     ctx, dw = hx.setup(w)
     r = dw.recall
     got = []
