@@ -135,7 +135,8 @@ def test_gated_step_with_recall_head(torch, ctxlen):
     st.close()
 
 
-def test_step_recall_split_plain_and_graph(torch):
+@pytest.mark.parametrize("B", [1, 16, 64])
+def test_step_recall_split_plain_and_graph(torch, B):
     """The step splits the head's first layer: h_{t-1} and E(x_t) in a kernel
     that starts with the step (beside the Local launches in the graph, first
     on one stream otherwise), h^L_t after the last Local launch. A rank of the
@@ -146,8 +147,9 @@ def test_step_recall_split_plain_and_graph(torch):
     steps agree bit for bit."""
     from gated_local_full_b200.runtime import DecodeStep
     from gated_local_full_b200 import oda
-    # a step of enough layers for the split (batch 16, hidden 2048, 6144 -> 4096)
-    w = synth.custom("recall_split", layers=oda.RECALL_SPLIT_MIN_LAYERS, batch=16, t0=[300],
+    # a step of enough layers for the split (hidden 2048, 6144 -> 4096; batch
+    # widths 16 and 64)
+    w = synth.custom("recall_split", layers=oda.RECALL_SPLIT_MIN_LAYERS, batch=B, t0=[300],
                      hq=16, hkv=8, window=128, recall=True, hidden=2048, recall_hidden=4096)
     ctx, dw = hx.setup(w)
     r = dw.recall
