@@ -442,22 +442,42 @@ attn_kernel(const AttnArgs a) {
   // Each warp walks its CTA's tile range with stride W. In the aligned
   // partition a long segment keeps its last ODA_POOL_PERCENT % of tiles in a
   // pool: a warp that finishes its static share takes pool tiles one at a
-  // time from the segment's counter (two grabs kept in flight), so warps
-  // that stream faster take more and the segment's CTAs finish together.
-  // The pool counters are scratch: they are touched only after the wait.
+  // time from the segment's counter, so warps that stream faster take more
+  // and the segment's CTAs finish together. Grabs run ahead of use without
+  // waiting on a round trip: three tiles before the end of its static share
+  // a warp takes three counter values, one tile later it looks up the first
+  // two tiles' blocks, and from then on each grab's counter value is looked
+  // up one tile after it was taken and used one tile after that. The pool
+  // counters are scratch: they are touched only after the wait.
   Cursor prod;
   prod.k = prod.i = prod.g = prod.nt = prod.s1 = 0;
   int seg_b = 0, seg_g0 = 0, seg_nt = 0, seg_s0 = 0, sigma0 = 0;
   int pool0 = 0;                             // first pool tile (relative); == nt: no pool
   bool use_pool = false;
-  int q0 = 0, q1 = 0, qb0 = -1, qb1 = -1;    // lane 0: grabbed pool tiles, blocks
-  auto grab = [&](int& q, int& qb) {         // lane 0 only, after the dependency wait
-    q = pool0 + atomicAdd(&a.dyn[sigma0], 1);
+  int q0 = 0, q1 = 0, qb0 = -1, qb1 = -1;    // lane 0: the next two pool tiles, their blocks
+  int gp = 0;                                // lane 0: a counter value not looked up yet
+  int pool_state = 0;                        // warp-uniform: 0 none, 1 gfirst taken, 2 armed
+  auto lookup = [&](int q) -> int {          // lane 0: the block of pool tile q
     // (the pool belongs to the first segment, row sigma0 / hkv)
-    qb = (!RING && q < seg_nt)
-             ? a.block_table[(long long)seg_b * a.max_blocks +
-                             (rowlo[sigma0 / a.hkv] - 1) / ODA_TILE + q]
-             : -1;
+    return (!RING && q < seg_nt)
+               ? a.block_table[(long long)seg_b * a.max_blocks +
+                               (rowlo[sigma0 / a.hkv] - 1) / ODA_TILE + q]
+               : -1;
+  };
+  auto prime_pool = [&]() {                  // warp, after the dependency wait, per refill
+    if (pool_state == 0 && prod.k + 3 * W >= hi) {
+      if (lane == 0) gp = atomicAdd(&a.dyn[sigma0], 3);
+      pool_state = 1;
+    } else if (pool_state == 1 && prod.k + 2 * W >= hi) {
+      if (lane == 0) {
+        q0 = pool0 + gp;
+        q1 = q0 + 1;
+        gp += 2;
+        qb0 = lookup(q0);
+        qb1 = lookup(q1);
+      }
+      pool_state = 2;
+    }
   };
 
   // Block ids of the producer's next 32 tiles of the current row, one per
@@ -473,14 +493,16 @@ attn_kernel(const AttnArgs a) {
       normalize(rowstart, a.hkv, hi, warp, prod);
       return true;
     }
-    if (!use_pool) return false;
+    if (!use_pool || pool_state < 2) return false;
     const int rel = __shfl_sync(0xffffffffu, q0, 0);
     blk = __shfl_sync(0xffffffffu, qb0, 0);
     if (rel >= seg_nt) return false;
     if (lane == 0) {
       q0 = q1;
       qb0 = qb1;
-      grab(q1, qb1);
+      q1 = pool0 + gp;                       // taken one tile ago
+      qb1 = lookup(q1);                      // needed one tile from now
+      gp = atomicAdd(&a.dyn[sigma0], 1);
     }
     k = seg_s0 + rel; i = prod.i; g = prod.g; nt = seg_nt;
     return true;
@@ -604,10 +626,6 @@ attn_kernel(const AttnArgs a) {
 #pragma unroll
     for (int h = 0; h < G; ++h) qraw[h] = sq[h * LPR + li];
     tpre = st_t[0];
-  }
-  if (use_pool && lane == 0) {       // after the first copies are in flight
-    grab(q0, qb0);
-    grab(q1, qb1);
   }
   __syncwarp();
   int consumed = 0;
@@ -827,6 +845,7 @@ attn_kernel(const AttnArgs a) {
       // refill the stage just consumed
       if (!prod_done && !aborted) {
         int k, i, g, nt, blk;
+        if (use_pool) prime_pool();
         if (next_tile(k, i, g, nt, blk)) {
           issue(k, i, g, nt, blk, stage);
           ++issued;
