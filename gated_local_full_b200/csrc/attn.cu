@@ -226,6 +226,7 @@ attn_kernel(const AttnArgs a) {
   uint4* sq = reinterpret_cast<uint4*>(rml + 32 * G);   // [QCH] the current segment's queries
   int* st_t = reinterpret_cast<int*>(sq + QCH);         // cluster mode: the row's t
   int* rowlo = st_t + 4;                                // paged: [max_batch] first position read
+  int* spool = rowlo + a.max_batch;                     // [W][4] pool grabs ahead (lane 0)
 
   const int tid = threadIdx.x;
   const int lane = tid & 31;
@@ -454,9 +455,11 @@ attn_kernel(const AttnArgs a) {
   int seg_b = 0, seg_g0 = 0, seg_nt = 0, seg_s0 = 0, sigma0 = 0;
   int pool0 = 0;                             // first pool tile (relative); == nt: no pool
   bool use_pool = false;
-  int q0 = 0, q1 = 0, qb0 = -1, qb1 = -1;    // lane 0: the next two pool tiles, their blocks
-  int gp = 0;                                // lane 0: a counter value not looked up yet
-  int pool_state = 0;                        // warp-uniform: 0 none, 1 gfirst taken, 2 armed
+  // lane 0: the next pool tile and its block in registers; the one after it,
+  // its block and a counter value not looked up yet in spool[warp] (q1, qb1, gp)
+  int q0 = 0, qb0 = -1;
+  int* sp = spool + 4 * warp;
+  int pool_state = 0;                        // warp-uniform: 0 none, 1 counters taken, 2 armed
   auto lookup = [&](int q) -> int {          // lane 0: the block of pool tile q
     // (the pool belongs to the first segment, row sigma0 / hkv)
     return (!RING && q < seg_nt)
@@ -466,15 +469,16 @@ attn_kernel(const AttnArgs a) {
   };
   auto prime_pool = [&]() {                  // warp, after the dependency wait, per refill
     if (pool_state == 0 && prod.k + 3 * W >= hi) {
-      if (lane == 0) gp = atomicAdd(&a.dyn[sigma0], 3);
+      if (lane == 0) sp[2] = atomicAdd(&a.dyn[sigma0], 3);
       pool_state = 1;
     } else if (pool_state == 1 && prod.k + 2 * W >= hi) {
       if (lane == 0) {
-        q0 = pool0 + gp;
-        q1 = q0 + 1;
-        gp += 2;
+        const int g3 = sp[2];
+        q0 = pool0 + g3;
         qb0 = lookup(q0);
-        qb1 = lookup(q1);
+        sp[0] = q0 + 1;
+        sp[1] = lookup(q0 + 1);
+        sp[2] = g3 + 2;
       }
       pool_state = 2;
     }
@@ -498,11 +502,12 @@ attn_kernel(const AttnArgs a) {
     blk = __shfl_sync(0xffffffffu, qb0, 0);
     if (rel >= seg_nt) return false;
     if (lane == 0) {
-      q0 = q1;
-      qb0 = qb1;
-      q1 = pool0 + gp;                       // taken one tile ago
-      qb1 = lookup(q1);                      // needed one tile from now
-      gp = atomicAdd(&a.dyn[sigma0], 1);
+      q0 = sp[0];
+      qb0 = sp[1];
+      const int q1 = pool0 + sp[2];          // taken one tile ago
+      sp[0] = q1;
+      sp[1] = lookup(q1);                    // needed one tile from now
+      sp[2] = atomicAdd(&a.dyn[sigma0], 1);
     }
     k = seg_s0 + rel; i = prod.i; g = prod.g; nt = seg_nt;
     return true;
@@ -583,7 +588,7 @@ attn_kernel(const AttnArgs a) {
       hi = seg_s0 + (int)(((long long)(part_al + 1) * pool0) / nparts_al);
     }
     use_pool = pool0 < seg_nt;
-    q0 = q1 = seg_nt;
+    q0 = seg_nt;
     if (!early) {
       if (warp == 0) load_q(seg_b, seg_g0, CL);
       q_loaded = true;
@@ -1188,6 +1193,7 @@ size_t smem_bytes_wn(int max_batch) {
   s += 16 + (size_t)(G * D + 32 * G) * 4;     // cluster mode: pushed accumulators, (m, l)
   s += (size_t)G * D * sizeof(T) + 16;          // the segment's queries, t
   s += (size_t)max_batch * 4;                   // first position read per row (paged)
+  s += (size_t)W * 4 * 4;                       // pool grabs ahead, per warp
   return (s + 127) & ~(size_t)127;
 }
 
