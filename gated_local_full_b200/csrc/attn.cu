@@ -395,7 +395,9 @@ attn_kernel(const AttnArgs a) {
   const int P = sinfo[2];
   const bool aligned = sinfo[3] != 0;
   int lo = sinfo[4], hi = sinfo[5];
-  const int pbase_al = sinfo[6], nparts_al = sinfo[7], part_al = sinfo[8], vcta = sinfo[9];
+  const int pbase_al = sinfo[6], nparts_al = sinfo[7], part_al = sinfo[8];
+  // partial slot of this CTA: its segment's own range in the aligned partition
+  const int vcta = (sinfo[3] && !CL) ? pbase_al + part_al : sinfo[9];
   const int cta = (int)blockIdx.x;
   // Cluster mode: each rank owns G*D/cs output elements of the segment. A
   // rank merges its warps' states (or takes an empty one) and pushes, with

@@ -162,7 +162,10 @@ __device__ __forceinline__ void plan_cta(int cta, const PlanHead& h, const int* 
     }
     const int nt = (rowstart[r0 + 1] - rowstart[r0]) / hkv;
     const int n = (rowcs[r0 + 1] - rowcs[r0]) / hkv;
-    const int g = (cta - rowcs[r0]) / n, part = cta - rowcs[r0] - g * n;
+    // the row's n * hkv CTAs interleave its segments (CTA l of the row works
+    // segment l % hkv): the CTAs dispatched last, which start and stream
+    // later, are spread over every segment, whose pools absorb them
+    const int g = (cta - rowcs[r0]) % hkv, part = (cta - rowcs[r0]) / hkv;
     const int s0 = rowstart[r0] + g * nt;
     if ((unsigned)nt < (1u << 31) / (unsigned)(n + 1)) {
       out[0] = s0 + (int)(((unsigned)part * (unsigned)nt) / (unsigned)n);
