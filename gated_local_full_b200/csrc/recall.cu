@@ -86,6 +86,14 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// L2 prefetch of one tile of a tensor map (no completion to wait for).
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y)
+               : "memory");
+}
+
 // Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
 // 1024 bytes apart (SBO), leading offset unused (1), descriptor version 1.
 __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t addr) {
@@ -503,6 +511,10 @@ recall_cluster_kernel(const __grid_constant__ CUtensorMap tm_w1,
       mbar_arrive_expect_tx(fb, tx);
       tma_load_2d(smem_addr(sa + (size_t)i * A_STAGE_BYTES), &tm_w1, (kb0 + i) * BK, mt * BM, fb);
     }
+    // the share's W1 tiles beyond the stages go to L2, so that the loads
+    // which refill the stages after the wait find them there
+    if (a.early)
+      for (int i = pre; i < kb1 - kb0; ++i) tma_prefetch_2d(&tm_w1, (kb0 + i) * BK, mt * BM);
   }
   auto load_owner_weights = [&]() {
     for (int rl = tid - 64; rl >= 0 && rl < RP; rl += 128) {
@@ -673,10 +685,17 @@ recall_cluster_kernel(const __grid_constant__ CUtensorMap tm_w1,
     }
     epi_bar();
   }
+  // Only the batch's columns are reduced (B rounded up to a power of two, at
+  // most N, itself a power of two here; the tile's other columns are
+  // padding): TPN threads per column, each taking rows t0, t0 + TPN, ... of
+  // the owned ones.
+  int NB = 1;
+  while (NB < a.B) NB <<= 1;
+  const int TPN = BM / NB;                                // threads per batch column
+  const int TPR = TPN < RP ? TPN : RP;                    // of which hold rows
   if (warp >= 2) {
     const int j = tid - 64;                               // 0..127
-    const int TPN = BM / N;                               // threads per batch row
-    const int n = j % N, t0 = j / N;
+    const int n = j % NB, t0 = j / NB;
     float s = 0.f;
     // fixed order; unrolled so that the rows' GELU chains overlap
 #pragma unroll 4
@@ -698,11 +717,10 @@ recall_cluster_kernel(const __grid_constant__ CUtensorMap tm_w1,
   __syncthreads();
   if (warp >= 2) {
     const int j = tid - 64;
-    const int TPN = BM / N;
-    if (j < N) {
+    if (j < NB) {
       float s = 0.f;
 #pragma unroll 8
-      for (int t2 = 0; t2 < TPN; ++t2) s += red[t2 * N + j];
+      for (int t2 = 0; t2 < TPR; ++t2) s += red[t2 * NB + j];
       a.spart[(size_t)blockIdx.x * N + j] = s;
     }
   }
