@@ -39,7 +39,8 @@ def _recall_oracle(w, step=0, W1=None, b1=None):
 
 
 SHAPES = [(16, 2048, 4096), (1, 2048, 4096), (17, 64, 128), (5, 192, 384), (256, 128, 256),
-          (33, 2048, 4096)]
+          (33, 2048, 4096), (2, 64, 128), (3, 192, 384), (4, 2048, 4096), (1, 1024, 8192),
+          (2, 4096, 1024)]
 
 
 @pytest.mark.parametrize("B,H,hidden", SHAPES, ids=[f"B{b}_H{h}_hid{n}" for b, h, n in SHAPES])
@@ -135,7 +136,7 @@ def test_gated_step_with_recall_head(torch, ctxlen):
     st.close()
 
 
-@pytest.mark.parametrize("B", [1, 16, 64])
+@pytest.mark.parametrize("B", [1, 2, 16, 64])
 def test_step_recall_split_plain_and_graph(torch, B):
     """The step splits the head's first layer: h_{t-1} and E(x_t) in a kernel
     that starts with the step (beside the Local launches in the graph, first
@@ -176,3 +177,4 @@ def test_step_recall_split_plain_and_graph(torch, B):
     alone = s.cpu().numpy().astype(np.float64)
     hx.assert_close(alone, ref, SCORE_ATOL, SCORE_RTOL, "standalone scores")
     np.testing.assert_allclose(alone, got[0], rtol=1e-5, atol=1e-5)
+
