@@ -13,8 +13,9 @@
 // denormal score is above theta = 0); NaN never compares greater. Flagged ids
 // are written in ascending order and the tail of idx is -1.
 //
-// The step graph creates its conditional handle with the default value 0
-// applied at every launch, so the gate sets it only when a row is flagged.
+// The gate sets the step graph's condition on every launch (1 when a row is
+// flagged, else 0): the handle carries no default, whose reset at each graph
+// launch measured slower than this store.
 #pragma once
 
 #include "oda_internal.cuh"
@@ -56,7 +57,7 @@ __device__ __forceinline__ void gate_block(const float* scores, float theta, int
   }
   if (tid == 0) {
     *count = total;
-    if (set_cond && total > 0) cudaGraphSetConditional(cond, 1u);
+    if (set_cond) cudaGraphSetConditional(cond, total > 0 ? 1u : 0u);
   }
 }
 
@@ -77,7 +78,7 @@ __device__ __forceinline__ void gate_warp(float v, int B, float theta, uint8_t* 
   }
   if (lane == 0) {
     *count = total;
-    if (set_cond && total > 0) cudaGraphSetConditional(cond, 1u);
+    if (set_cond) cudaGraphSetConditional(cond, total > 0 ? 1u : 0u);
   }
 }
 

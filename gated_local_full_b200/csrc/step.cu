@@ -166,13 +166,12 @@ oda_status oda_step_graph_create(oda_ctx* ctx, const oda_step_desc* d, oda_graph
     cudaGraph_t cap = nullptr;
     const cudaGraphNode_t* deps = nullptr;
     size_t ndeps = 0;
-    // the condition is 0 at the start of every launch; the gate sets it to 1
-    // when it flags a row
+    // the gate sets the condition on every launch (1 when it flags a row,
+    // else 0), so the handle needs no default applied at each launch
     cudaGraphConditionalHandle handle = 0;
     bool ok = cudaStreamGetCaptureInfo(st, &cs, nullptr, &cap, &deps, &ndeps) == cudaSuccess &&
               cs == cudaStreamCaptureStatusActive &&
-              cudaGraphConditionalHandleCreate(&handle, cap, 0, cudaGraphCondAssignDefault) ==
-                  cudaSuccess;
+              cudaGraphConditionalHandleCreate(&handle, cap, 0, 0) == cudaSuccess;
     oda_status ps =
         ok ? pre_part(ctx, d, st, st3, fork, join, (unsigned long long)handle, true) : ODA_ERR_CUDA;
     cudaGraphNode_t cond_node = nullptr;
